@@ -1,0 +1,309 @@
+#!/usr/bin/env python3
+"""Benchmark of the routed-MoE layer on B200: GLM-5.2-shaped single-layer decode.
+
+Workload (one "step" = one pass of the whole layer over one batch):
+  T = 1 token, hidden 6144, 256 routed experts in 8 groups (topk_group 4),
+  top-8, expert intermediate 2048, packed int4 weights with fp32 per-row
+  scales (18,915,328 B per expert), one shared expert of the same shape,
+  fp32 router N(0, 0.02^2), bias N(0, 0.1^2), rsf 2.5; all 257 experts
+  resident in HBM (4.86 GB); every step routes a different seeded bf16 N(0,1)
+  token, and the L2 cache is flushed (a 512 MB write) between timed steps.
+
+Arms:
+  default           the CUDA path through the C ABI (moe_layer_forward)
+  --impl reference  the CPU oracle (plain C, OpenMP) on the host cores, on a
+                    bounded sample of the same workload
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): replicas only, each rank
+runs its own copy of the layer; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "routed-MoE layer tokens/s; int4 expert-weight GB/s vs ~8 TB/s HBM peak"
+WORKLOAD = ("GLM-5.2-shaped single-layer decode: T=1, hidden 6144, 256 routed experts "
+            "(8 groups, topk_group 4), top-8, intermediate 2048, packed int4 + fp32 row scales, "
+            "1 shared expert, rsf 2.5")
+NOMINAL_HBM_GBS = 8000.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--pool", type=int, default=512, help="distinct seeded tokens cycled through")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(sh, seconds: float, first_token: int = 0, max_tokens: int | None = None):
+    """Time the CPU oracle's full layer on successive seeded tokens for ~`seconds`."""
+    from oracle import oracle as O
+    from tests.helpers import oracle_experts
+
+    W = synth.router_weight(sh)
+    b = synth.router_bias(sh)
+    shared = oracle_experts(sh, [0], shared=True)
+    total, n, t = 0.0, 0, first_token
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    while (total < seconds or n == 0) and (max_tokens is None or n < max_tokens):
+        x = synth.hidden_states(sh, tokens=[t])
+        idx, _, _, _ = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+        routed = oracle_experts(sh, np.unique(idx))
+        t0 = time.perf_counter()
+        O.layer_forward(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf, routed, shared)
+        total += time.perf_counter() - t0
+        n += 1
+        t += 1
+    return dict(value=n * sh.T / total, unit="tokens/s", cores=threads, kind="oracle",
+                sample=f"{n} decode tokens (T=1 layer calls, each routed afresh), "
+                       f"{total:.1f} s of oracle time; weight generation excluded"), n, total
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sh = synth.CONFIGS["decode"]
+    # one step = one token's full layer on the CPU oracle; warm-up and timed
+    # tokens are capped so that the whole run stays within a few minutes
+    if args.warmup > 0:
+        oracle_sample(sh, 0.0, first_token=10_000, max_tokens=min(args.warmup, 3))
+    cb, n, total = oracle_sample(sh, 120.0, first_token=0, max_tokens=args.steps)
+    value = cb["value"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / max(n, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4xint8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "T": sh.T, "cpu": "host cores"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CUDA arm
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_mixture_experts_sigmoid_b200 import moe
+    from tests.gpu_fixtures import device_layer, to_dev_bf16
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    sh = synth.CONFIGS["decode"]
+    dev = device_layer(sh)
+    routed, shared = dev["routed"], dev["shared"]
+    T, H = sh.T, sh.H
+    pool = synth.hidden_states(sh, tokens=range(rank * args.pool, (rank + 1) * args.pool))
+    xs = to_dev_bf16(pool)  # [pool, H]: one distinct token per step, cycled
+    out = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(T, sh.top_k, dtype=torch.int32, device="cuda")
+    wts = torch.empty(T, sh.top_k, dtype=torch.float32, device="cuda")
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(T, dev["cfg"], routed, shared))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        moe.moe_layer_forward(xs[i % args.pool:i % args.pool + 1], dev["W"], dev["bias"], dev["cfg"],
+                              routed, shared, out, ws, idx, wts)
+
+    for i in range(args.warmup):
+        step(i)
+        flush.zero_()
+    torch.cuda.synchronize()
+    if moe.moe_workspace_status(ws) != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    # ---- device-resident timing: per-step events, L2 flushed between steps
+    n_ev = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    L = moe.lib()
+    launches0 = L.moe_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    L.moe_profile_enable(1)
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(args.warmup + i)
+            stops[i].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    launches = L.moe_launch_count() - launches0
+    import ctypes
+    kms, kn = ctypes.c_double(0), ctypes.c_int(0)
+    L.moe_profile_read(ctypes.byref(kms), ctypes.byref(kn))
+    L.moe_profile_enable(0)
+    dev_ms = sum(s.elapsed_time(e) for s, e in zip(starts, stops))
+    t_max = torch.tensor([dev_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    dev_ms = float(t_max.item())
+    if moe.moe_workspace_status(ws) != 0:
+        raise RuntimeError("device status error during timing")
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    x_host = torch.from_numpy(pool.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    e2e_steps = min(args.steps, 1000)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_stops = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        j = (args.warmup + i) % args.pool
+        e_starts[i].record(stream)
+        x_dev.copy_(x_host[j:j + 1], non_blocking=True)
+        moe.moe_layer_forward(x_dev, dev["W"], dev["bias"], dev["cfg"], routed, shared, out, ws)
+        out_host.copy_(out, non_blocking=True)
+        e_stops[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_stops))
+    t_e2e = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t_e2e.item())
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    ms_step = dev_ms / args.steps
+    tok_s = world * T * args.steps / (dev_ms / 1e3)
+    U = sh.top_k  # T = 1: every step touches top_k distinct routed experts
+    expert_bytes = (U + 1) * sh.expert_bytes()
+    layer_bytes = expert_bytes + sh.router_bytes()
+    hbm_peak, peak_kind = peaks()
+    # dominant kernel: the routed up/gate streaming kernel (2/3 of the routed bytes)
+    dom_bytes = U * (2 * sh.matrix_bytes(synth.GATE) + 2 * 4 * sh.I)
+    dom_ms = kms.value / max(kn.value, 1)
+    dom_gbs = dom_bytes / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int4xint8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": T, "H": H, "I": sh.I, "E": sh.E, "top_k": sh.top_k,
+                   "parallelism": f"replicas x{world}", "l2": "flushed between timed steps",
+                   "tokens_cycled": args.pool},
+        "expert_weight_GBps": expert_bytes / (ms_step / 1e3) / 1e9,
+        "layer_GBps": layer_bytes / (ms_step / 1e3) / 1e9,
+        "layer_bytes_per_step": layer_bytes,
+        "frac_of_8TBps": layer_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "kernel": "routed expert up/gate streaming kernel",
+                     "achieved": dom_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": None,
+                     "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
+        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "wall_s_timed_region": wall,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        cb, _, _ = oracle_sample(sh, args.cpu_seconds)
+        line["cpu_baseline"] = cb
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -25,8 +25,10 @@ def build(force: bool = False) -> str:
         os.path.getmtime(SO) >= os.path.getmtime(s) for s in (SRC, HDR))
     if force or not fresh:
         os.makedirs(BUILD, exist_ok=True)
+        tmp = f"{SO}.{os.getpid()}.tmp"
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
-                               "-fopenmp", "-fPIC", "-shared", SRC, "-o", SO, "-lm"])
+                               "-fopenmp", "-fPIC", "-shared", SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, SO)
     return SO
 
 

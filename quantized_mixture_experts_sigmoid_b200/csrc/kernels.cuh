@@ -1,0 +1,53 @@
+// Launch wrappers of the library's kernels (internal; the C ABI is in moe.h).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Raises a kernel's dynamic shared-memory cap to `bytes` (once per kernel and device).
+cudaError_t ensure_smem(const void* kernel, size_t bytes);
+
+// Adds n to the process-wide count of kernels this library launched.
+void count_launch(int n = 1);
+
+// Returns e after counting one launch when it succeeded.
+inline cudaError_t counted(cudaError_t e) {
+    if (e == cudaSuccess) count_launch(1);
+    return e;
+}
+
+cudaError_t launch_router_logits(const uint16_t* x, int T, int H, const float* w, int E,
+                                 float* logits, cudaStream_t st);
+cudaError_t launch_router_select(const float* logits, int T, const float* bias,
+                                 const moe_router_cfg& c, int32_t* idx, float* w, int32_t* status,
+                                 cudaStream_t st);
+
+cudaError_t launch_union(const int32_t* idx, int T, int K, int E, int32_t* n_unique, int32_t* uniq,
+                         int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot, int32_t* counts,
+                         int32_t* status, cudaStream_t st);
+
+cudaError_t launch_q8_0(const void* v, bool bf16, long rows, int n, int8_t* q, float* d,
+                        cudaStream_t st);
+
+// Union descriptor of one expert pass.  uniq == nullptr: dense mode (expert 0, pair p = token p).
+struct UnionView {
+    const int32_t* n_unique;
+    const int32_t* uniq;
+    const int32_t* offsets;
+    const int32_t* pair_tok;
+    const int32_t* pair_slot;
+    int max_unique;  // grid bound (device value n_unique <= max_unique)
+};
+
+// up/gate + SwiGLU + Q8_0(h) for every pair; qh [P][I], dh [P][I/32] by pair index.
+cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
+                                  const UnionView& un, int8_t* qh, float* dh, cudaStream_t st);
+// down rows for every pair, written to y_pairs[tok][slot][:].
+cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
+                               int top_k, const UnionView& un, float* y_pairs, cudaStream_t st);
+
+cudaError_t launch_combine(const float* y, const float* w, const float* shared_y, int T, int K,
+                           int H, void* out, int out_dtype, cudaStream_t st);
+
+}  // namespace moe

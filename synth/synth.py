@@ -116,7 +116,9 @@ def build_host(force: bool = False) -> str:
     src = os.path.join(HERE, "synth_host.c")
     if force or not _newer(HOST_SO, src):
         os.makedirs(BUILD, exist_ok=True)
-        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", src, "-o", HOST_SO])
+        tmp = f"{HOST_SO}.{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", src, "-o", tmp])
+        os.replace(tmp, HOST_SO)
     return HOST_SO
 
 
@@ -124,9 +126,11 @@ def build_gpu(force: bool = False) -> str:
     src = os.path.join(HERE, "synth_gpu.cu")
     if force or not _newer(GPU_SO, src):
         os.makedirs(BUILD, exist_ok=True)
+        tmp = f"{GPU_SO}.{os.getpid()}.tmp"
         subprocess.check_call([
             "nvcc", "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
-            "-Xcompiler", "-fPIC", "-shared", src, "-o", GPU_SO])
+            "-Xcompiler", "-fPIC", "-shared", src, "-o", tmp])
+        os.replace(tmp, GPU_SO)
     return GPU_SO
 
 
