@@ -46,6 +46,7 @@ typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
 #define MOE_ECUDA (-4)          /* a CUDA launch or copy failed */
 #define MOE_EDEVICE_TIMEOUT (-5) /* a bounded device-side wait gave up (see moe_workspace_status) */
 #define MOE_EDEVICE_INDEX (-6)  /* a kernel saw an out-of-range expert index (see moe_workspace_status) */
+#define MOE_ETOO_LARGE (-7)     /* the batch exceeds a fixed capacity (moe_route_noalloc) */
 
 /* Human-readable text of an MOE_* code (static string, never NULL). */
 const char* moe_strerror(int code);
@@ -118,6 +119,36 @@ size_t moe_route_workspace_bytes(int T, const moe_router_cfg* cfg);
 int moe_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
               const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w, void* ws,
               size_t ws_bytes, moe_stream_t stream);
+
+/* Capacity, in fp32 logits (T * n_expert), of moe_route_noalloc's built-in
+ * scratch: 65536 logits = 256 KiB of device memory on every GPU that loads
+ * the library, held until the process exits. */
+#define MOE_ROUTE_NOALLOC_MAX_LOGITS 65536
+
+/*
+ * moe_route without a workspace, for callers that cannot allocate device
+ * memory when they route: work recorded into a CUDA graph while a stream is
+ * being captured, inference-engine plugins whose enqueue step must not
+ * allocate, or latency-critical loops that cannot afford cudaMalloc's implicit
+ * device synchronisation.  The pages have no counterpart to this call; it is
+ * part of this library's interface only.
+ *
+ * Same arguments and results as moe_route minus ws / ws_bytes.  The logits
+ * scratch is a fixed array inside the library (MOE_ROUTE_NOALLOC_MAX_LOGITS
+ * floats); batches with T * n_expert above that return MOE_ETOO_LARGE and
+ * launch nothing.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before capturing a stream on the device.
+ *  - Every call in the process shares the one array per device and leaves its
+ *    logits there.  Calls whose kernels may overlap on the same device (on
+ *    different streams, or from different threads) race on it: order them.
+ *  - Unlike moe_route it records no device-side status word.
+ */
+int moe_route_noalloc(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
+                      const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w,
+                      moe_stream_t stream);
 
 /* ------------------------------------------------------------------ union */
 

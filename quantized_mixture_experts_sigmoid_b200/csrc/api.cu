@@ -179,6 +179,7 @@ const char* moe_strerror(int code) {
         case MOE_ECUDA: return "CUDA launch or copy failed";
         case MOE_EDEVICE_TIMEOUT: return "a bounded device-side wait gave up";
         case MOE_EDEVICE_INDEX: return "a kernel saw an expert index outside [0, E)";
+        case MOE_ETOO_LARGE: return "batch exceeds the fixed scratch capacity of moe_route_noalloc";
         default: return "unknown moe error code";
     }
 }

@@ -22,6 +22,8 @@ MOE_EUNSUPPORTED = -3
 MOE_ECUDA = -4
 MOE_EDEVICE_TIMEOUT = -5
 MOE_EDEVICE_INDEX = -6
+MOE_ETOO_LARGE = -7
+MOE_ROUTE_NOALLOC_MAX_LOGITS = 65536
 MOE_Q_INT2, MOE_Q_INT4, MOE_Q_INT8 = 2, 4, 8
 MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
 
@@ -85,7 +87,8 @@ _lib = None
 EXPORTS = ["moe_strerror", "moe_route_workspace_bytes", "moe_route", "moe_union",
            "moe_quantize_q8_0", "moe_expert_ffn_workspace_bytes", "moe_expert_ffn_q",
            "moe_combine", "moe_layer_workspace_bytes", "moe_layer_forward",
-           "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count"]
+           "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count",
+           "moe_route_noalloc"]
 
 
 def lib() -> ctypes.CDLL:
@@ -103,6 +106,7 @@ def lib() -> ctypes.CDLL:
     L.moe_route_workspace_bytes.argtypes = [i, vp]
     L.moe_route_workspace_bytes.restype = sz
     L.moe_route.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.moe_route_noalloc.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp]
     L.moe_union.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_quantize_q8_0.argtypes = [vp, i, i, i, vp, vp, vp]
     L.moe_expert_ffn_workspace_bytes.argtypes = [vp, i, i]
@@ -156,6 +160,14 @@ def moe_route(x, w_router, bias, cfg: RouterCfg, topk_idx, topk_w, ws, stream=No
     _ok("moe_route", lib().moe_route(_ptr(x), T, H, _ptr(w_router), _ptr(bias), ctypes.byref(cfg),
                                      _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
                                      _stream(stream)))
+
+
+def moe_route_noalloc(x, w_router, bias, cfg: RouterCfg, topk_idx, topk_w, stream=None):
+    """moe_route with the library's built-in logits scratch (no workspace, allocates nothing)."""
+    T, H = x.shape
+    _ok("moe_route_noalloc", lib().moe_route_noalloc(_ptr(x), T, H, _ptr(w_router), _ptr(bias),
+                                                     ctypes.byref(cfg), _ptr(topk_idx),
+                                                     _ptr(topk_w), _stream(stream)))
 
 
 def moe_union(topk_idx, E, n_unique, uniq, offsets, pair_tok, pair_slot, counts=None,
