@@ -105,6 +105,10 @@ struct LayerWs {
     float* dhs;
     float* y;
     float* ys;
+    // fused small-batch path only (T <= kFusedMaxTokens)
+    int32_t* pair_of;
+    uint8_t* qrec;
+    float* yf;
     size_t bytes;
 };
 
@@ -133,8 +137,57 @@ LayerWs carve_layer(void* ws, int T, const moe_router_cfg& c, const moe_experts&
         L.ys = cv.take<float>(static_cast<size_t>(T) * H);
     }
     L.y = cv.take<float>(P * H);
+    if (T <= kFusedMaxTokens) {
+        L.pair_of = cv.take<int32_t>(P);
+        L.qrec = cv.take<uint8_t>((P + T) * fused_record_bytes(I));
+        L.yf = cv.take<float>((P + T) * static_cast<size_t>(H));
+    }
     L.bytes = align_up(cv.off, 256);
     return L;
+}
+
+// The fused kernel takes small batches whose shared expert (if any) has the
+// routed experts' qtype and intermediate size.
+bool fused_params(FusedParams& f, const LayerWs& L, void* ws, const uint16_t* x, int T,
+                  const float* w_router, const float* bias, const moe_router_cfg& c,
+                  const moe_experts& r, const moe_experts* s, void* out, int out_dtype,
+                  int32_t* idx, float* w) {
+    if (T > kFusedMaxTokens) return false;
+    if (s && (s->qtype != r.qtype || s->inter != r.inter || s->hidden != r.hidden)) return false;
+    f = FusedParams{};
+    f.x = x;
+    f.T = T;
+    f.H = r.hidden;
+    f.I = r.inter;
+    f.E = c.n_expert;
+    f.G = c.n_group;
+    f.TG = c.topk_group;
+    f.K = c.top_k;
+    f.rsf = c.routed_scaling_factor;
+    f.w_router = w_router;
+    f.bias = bias;
+    f.routed = r;
+    if (s) f.shared = *s;
+    f.has_shared = s != nullptr;
+    f.out = out;
+    f.out_bf16 = out_dtype == MOE_OUT_BF16;
+    f.idx = idx;
+    f.w = w;
+    char* base = static_cast<char*>(ws);
+    f.status = reinterpret_cast<int32_t*>(base + kWsStatusOff);
+    f.sync = reinterpret_cast<FusedSync*>(base + kWsSyncOff);
+    f.ug_done = reinterpret_cast<int32_t*>(base + kWsUgDoneOff);
+    f.rb_done = reinterpret_cast<int32_t*>(base + kWsRbDoneOff);
+    f.logits = L.logits;
+    f.n_unique = L.n_unique;
+    f.uniq = L.uniq;
+    f.offsets = L.offsets;
+    f.pair_tok = L.pair_tok;
+    f.pair_slot = L.pair_slot;
+    f.pair_of = L.pair_of;
+    f.qrec = L.qrec;
+    f.y = L.yf;
+    return fused_geometry(f, r.qtype);
 }
 
 struct FfnWs {
@@ -306,6 +359,14 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
     const int H = routed->hidden, K = cfg->top_k, E = cfg->n_expert;
     int32_t* idx = topk_idx_out ? topk_idx_out : L.idx;
     float* w = topk_w_out ? topk_w_out : L.w;
+
+    FusedParams f;
+    if (fused_params(f, L, ws, x, T, w_router, bias, *cfg, *routed, shared, out, out_dtype, idx, w)) {
+        const bool timed = g_prof.begin(st);
+        rc = cuda_rc(launch_decode_fused(f, st));
+        if (timed) g_prof.end(st);
+        return rc;
+    }
 
     if ((rc = cuda_rc(launch_router_logits(x, T, H, w_router, E, L.logits, st)))) return rc;
     if ((rc = cuda_rc(launch_router_select(L.logits, T, bias, *cfg, idx, w, L.status, st)))) return rc;

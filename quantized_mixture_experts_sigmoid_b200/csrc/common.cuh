@@ -17,8 +17,9 @@ namespace moe {
 constexpr int kWarp = 32;
 constexpr int kQBlock = 32;  // Q8_0 block length
 
-// Device status word offsets inside a workspace (first 256 bytes are a header).
-constexpr size_t kWsHeader = 256;
+// Every workspace starts with a control header: the device status word at
+// offset 0, then the fused kernel's self-resetting counters.
+constexpr size_t kWsHeader = 8192;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -50,4 +50,63 @@ cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const fl
 cudaError_t launch_combine(const float* y, const float* w, const float* shared_y, int T, int K,
                            int H, void* out, int out_dtype, cudaStream_t st);
 
+// ------------------------------------------------------------ fused small-batch layer
+constexpr int kFusedMaxTokens = 4;
+
+// Control block at the start of every workspace (kWsHeader bytes, zero when idle).
+struct FusedSync {
+    int ticket;
+    int router_done;
+    int route_ready;
+    int exit_count;
+    int pad[12];
+};
+constexpr size_t kWsStatusOff = 0;
+constexpr size_t kWsSyncOff = 64;
+constexpr size_t kWsUgDoneOff = 128;                    // int[E + 1], E <= 1024
+constexpr size_t kWsRbDoneOff = kWsUgDoneOff + 4 * 1032; // int[n_dt], n_dt <= 16384 / 32 + 1
+static_assert(kWsRbDoneOff + 4 * 520 <= kWsHeader, "workspace header too small");
+
+struct FusedParams {
+    const uint16_t* x;
+    int T, H, I, E, G, TG, K;
+    float rsf;
+    const float* w_router;
+    const float* bias;
+    moe_experts routed;
+    moe_experts shared;
+    int has_shared;
+    void* out;
+    int out_bf16;
+    int32_t* idx;
+    float* w;
+    int32_t* status;
+    FusedSync* sync;
+    int32_t* ug_done;
+    int32_t* rb_done;
+    float* logits;
+    int32_t* n_unique;
+    int32_t* uniq;
+    int32_t* offsets;
+    int32_t* pair_tok;
+    int32_t* pair_slot;
+    int32_t* pair_of;
+    uint8_t* qrec;  // [(T*K + T)][rec_bytes] permuted Q8_0(h) records
+    float* y;       // [(T*K + T)][H] per-pair expert outputs (shared rows last)
+    int rec_bytes;
+    int nstage, stage_bytes, act_bytes, sr_down, dr, n_ugt, n_dt;
+    int rps;   // router rows per stage
+    int n_rt;  // router tickets
+    int nt;    // token capacity of the kernel instantiation (1 or kFusedMaxTokens)
+};
+
+// Bytes of one pair's Q8_0(h) record: two 16-byte planes per block, the block
+// scales and block sums, padded so records can be bulk-copied back to back.
+inline size_t fused_record_bytes(int I) { return (static_cast<size_t>(I) + I / 4 + 15) & ~size_t(15); }
+
+// Fills the geometry fields; false if the fused kernel cannot take this shape.
+bool fused_geometry(FusedParams& p, int qtype);
+size_t fused_smem_bytes(const FusedParams& p);
+cudaError_t launch_decode_fused(const FusedParams& p, cudaStream_t st);
+
 }  // namespace moe

@@ -13,6 +13,7 @@
 // summation order used here.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "router_select.cuh"
 
 namespace moe {
 namespace {
@@ -64,78 +65,14 @@ k_router_select(const float* __restrict__ logits, int T, const float* __restrict
                 float* __restrict__ topk_w, int32_t* status) {
     extern __shared__ float sm[];
     __shared__ int chosen[kSelectWarps][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * kSelectWarps + warp;
     if (t >= T) return;
     float* s = sm + static_cast<size_t>(warp) * 2 * E;
-    float* b = s + E;
     const float* lg = logits + static_cast<size_t>(t) * E;
-    for (int e = lane; e < E; e += 32) {
-        const double l = static_cast<double>(lg[e]);
-        const float sv = __double2float_rn(1.0 / (1.0 + exp(-l)));
-        s[e] = sv;
-        b[e] = __fadd_rn(sv, bias[e]);
-    }
-    __syncwarp();
-    const int gsz = E / G;
-    // group score: sum of the two largest biased scores (lane g owns group g)
-    float gs = -INFINITY;
-    if (lane < G) {
-        float v1 = -INFINITY, v2 = -INFINITY;
-        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
-            const float v = b[e];
-            if (v > v1) {
-                v2 = v1;
-                v1 = v;
-            } else if (v > v2) {
-                v2 = v;
-            }
-        }
-        gs = __fadd_rn(v1, v2);
-    }
-    uint32_t keep = 0;
-    for (int j = 0; j < TG; ++j) {
-        const bool ok = lane < G && !((keep >> lane) & 1u);
-        float v = ok ? gs : -INFINITY;
-        int i = ok ? lane : 0x7fffffff;
-        warp_argmax(v, i);
-        if (i >= G) {  // only reachable with NaN scores: keep indices in range, flag it
-            record_status(status, MOE_EDEVICE_INDEX);
-            i = 0;
-        }
-        keep |= 1u << i;
-    }
-    for (int k = 0; k < K; ++k) {
-        float best = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            if (!((keep >> (e / gsz)) & 1u)) continue;
-            const float v = b[e];
-            if (v > best) {  // ascending e within a lane: first of equals wins
-                best = v;
-                bi = e;
-            }
-        }
-        warp_argmax(best, bi);
-        if (bi >= E) {  // only reachable with NaN scores
-            record_status(status, MOE_EDEVICE_INDEX);
-            bi = 0;
-        }
-        if (lane == 0) {
-            chosen[warp][k] = bi;
-            b[bi] = -INFINITY;
-        }
-        __syncwarp();
-    }
-    if (lane == 0) {
-        float den = 0.0f;
-        for (int k = 0; k < K; ++k) den = __fadd_rn(den, s[chosen[warp][k]]);
-        for (int k = 0; k < K; ++k) {
-            const int e = chosen[warp][k];
-            topk_idx[static_cast<size_t>(t) * K + k] = e;
-            topk_w[static_cast<size_t>(t) * K + k] = __fmul_rn(__fdiv_rn(s[e], den), rsf);
-        }
-    }
+    select_token_warp([lg](int e) { return lg[e]; }, bias, E, G, TG, K, rsf, s, s + E,
+                      chosen[warp], topk_idx + static_cast<size_t>(t) * K,
+                      topk_w + static_cast<size_t>(t) * K, status);
 }
 
 }  // namespace

@@ -1,0 +1,93 @@
+// noaux_tc selection of one token by one warp (internal).
+//
+// [HN] "Show HN: 느린 컴퓨터에서 GLM 5.2 실행하기", section "구현된 주요 기능",
+// router bullet (DeepSeek-V3-style sigmoid router, noaux_tc,
+// routed_scaling_factor).  Reading: s = sigmoid(logit) in fp64 rounded once;
+// b = s + bias (for choosing only); group score = sum of the two largest b of
+// each contiguous group; keep topk_group groups; choose top_k experts by b
+// among kept groups; ties to the lower index; w = s / sum(s) * rsf with the
+// sum in slot order.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// s, b: this warp's shared-memory scratch of E floats each.  logit(e) returns
+// the fp32 logit of expert e.  Lane 0 writes idx[k], w[k] (k < K); chosen
+// (shared, >= K ints) receives the indices for every lane.
+template <typename LogitFn>
+__device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __restrict__ bias,
+                                                  int E, int G, int TG, int K, float rsf,
+                                                  float* s, float* b, int* chosen,
+                                                  int32_t* idx, float* w, int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    for (int e = lane; e < E; e += 32) {
+        const double l = static_cast<double>(logit(e));
+        const float sv = __double2float_rn(1.0 / (1.0 + exp(-l)));
+        s[e] = sv;
+        b[e] = __fadd_rn(sv, __ldg(bias + e));
+    }
+    __syncwarp();
+    const int gsz = E / G;
+    float gs = -INFINITY;
+    if (lane < G) {
+        float v1 = -INFINITY, v2 = -INFINITY;
+        for (int e = lane * gsz; e < (lane + 1) * gsz; ++e) {
+            const float v = b[e];
+            if (v > v1) {
+                v2 = v1;
+                v1 = v;
+            } else if (v > v2) {
+                v2 = v;
+            }
+        }
+        gs = __fadd_rn(v1, v2);
+    }
+    uint32_t keep = 0;
+    for (int j = 0; j < TG; ++j) {
+        const bool ok = lane < G && !((keep >> lane) & 1u);
+        float v = ok ? gs : -INFINITY;
+        int i = ok ? lane : 0x7fffffff;
+        warp_argmax(v, i);
+        if (i >= G) {  // only reachable with NaN scores: keep indices in range, flag it
+            record_status(status, MOE_EDEVICE_INDEX);
+            i = 0;
+        }
+        keep |= 1u << i;
+    }
+    for (int k = 0; k < K; ++k) {
+        float best = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            if (!((keep >> (e / gsz)) & 1u)) continue;
+            const float v = b[e];
+            if (v > best) {  // ascending e within a lane: first of equals wins
+                best = v;
+                bi = e;
+            }
+        }
+        warp_argmax(best, bi);
+        if (bi >= E) {  // only reachable with NaN scores
+            record_status(status, MOE_EDEVICE_INDEX);
+            bi = 0;
+        }
+        if (lane == 0) {
+            chosen[k] = bi;
+            b[bi] = -INFINITY;
+        }
+        __syncwarp();
+    }
+    if (lane == 0) {
+        float den = 0.0f;
+        for (int k = 0; k < K; ++k) den = __fadd_rn(den, s[chosen[k]]);
+        for (int k = 0; k < K; ++k) {
+            const int e = chosen[k];
+            idx[k] = e;
+            w[k] = __fmul_rn(__fdiv_rn(s[e], den), rsf);
+        }
+    }
+    __syncwarp();
+}
+
+}  // namespace moe

@@ -29,12 +29,20 @@ SHAPES = {
                                      topk_group=2, top_k=5, qtype=8),
     "crowded_int2": synth.LayerShape("crowded_int2", T=100, H=544, I=288, E=16, n_group=4,
                                      topk_group=2, top_k=5, qtype=2),
+    # small batches take the fused persistent kernel: ragged shapes, T = 2 and 3
+    "fused_ragged": synth.LayerShape("fused_ragged", T=3, H=544, I=288, E=48, n_group=6, topk_group=3,
+                                     top_k=5),
+    "fused_ragged_int2": synth.LayerShape("fused_ragged_int2", T=2, H=576, I=160, E=64, n_group=8,
+                                          topk_group=2, top_k=6, qtype=2),
+    "fused_ragged_int8": synth.LayerShape("fused_ragged_int8", T=4, H=544, I=288, E=48, n_group=6,
+                                          topk_group=3, top_k=5, qtype=8),
     "decode": synth.CONFIGS["decode"],
     "verify": synth.CONFIGS["verify"],
     "verify_int8": synth.CONFIGS["verify_int8"],
     "decode_int2": synth.CONFIGS["decode"].with_(qtype=2, name="decode_int2"),
 }
-SMALL = ["tiny", "ragged", "crowded", "crowded_int8", "crowded_int2"]
+SMALL = ["tiny", "ragged", "crowded", "crowded_int8", "crowded_int2", "fused_ragged",
+         "fused_ragged_int2", "fused_ragged_int8"]
 FULL = ["decode", "verify", "verify_int8", "decode_int2"]
 
 _cache = {}
@@ -267,3 +275,23 @@ def test_union_path_equals_per_token_path_on_gpu():
     for t in (0, 17, 99):
         of_one, _, _, _ = run_layer(sh, dev, x[t:t + 1])
         assert np.array_equal(of_one.view(np.uint32), of_batch[t:t + 1].view(np.uint32))
+
+
+def test_layer_forward_repeated_calls_reuse_workspace():
+    # the fused kernel's counters live in the workspace and reset themselves:
+    # many calls in a row on one workspace give the same, correct result
+    sh, dev = layer("decode")
+    x, W, b = layer_inputs(sh)
+    xd = to_dev_bf16(x)
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
+    outs = []
+    for i in range(20):
+        out = torch.empty(sh.T, sh.H, dtype=torch.float32, device="cuda")
+        moe.moe_layer_forward(xd, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert moe.moe_workspace_status(ws) == 0
+    first = outs[0].cpu().numpy()
+    for o in outs[1:]:
+        assert np.array_equal(o.cpu().numpy().view(np.uint32), first.view(np.uint32))
+    check_layer(sh, dev, x, W, b)
