@@ -23,10 +23,13 @@
 //      router rows | shared up/gate tiles | routed up/gate tiles |
 //      shared down tiles | routed down tiles
 // so every dependency points to an earlier ticket and every CTA sees its
-// stages in that order.  The CTA that finishes the last router row runs the
-// noaux_tc selection and the batch union for the whole batch (all consumer
-// threads, rank-based) and publishes them; producers that need the routing
-// wait for it.  An up/gate tile is 32 rows of h for one expert; its epilogue
+// stages in that order.  After its last router row a producer queues a
+// zero-byte route marker; at the marker the consumers wait until every logit
+// of the batch has been counted, then compute the noaux_tc selection and the
+// batch union themselves (all consumer threads, rank-based, in shared memory:
+// every CTA reaches the same result) and hand it to their producer through an
+// mbarrier.  Routing therefore costs one global round trip (the logit count)
+// rather than a publish by one CTA and a read-back by all.  An up/gate tile is 32 rows of h for one expert; its epilogue
 // writes Q8_0(h) as a pre-permuted activation record.  A down tile waits for
 // its expert's h tiles, then copies the records of its pairs next to its
 // weight stages.  The CTA that completes a row block of the output combines
@@ -63,6 +66,10 @@ constexpr int kMaxDownRowsPerWarp = 4;
 constexpr int kActSlots = 2;
 constexpr int kTaskSlots = 2;
 constexpr int kScaleBytes = 256;     // room after each stage for its rows' fp32 scales
+// Copies a producer keeps in flight.  Enough to cover HBM latency at full
+// bandwidth; more only lengthens the memory queues, and every other request
+// (logits, counters, instruction fetches) then waits behind them.
+constexpr int kMaxInflight = 2;
 constexpr int kRegChunksUg = 6;      // NT = 1: blocks of x per lane held in registers (H <= 6144)
 constexpr int kRegChunksDown = 2;    // NT = 1: blocks of h per lane held in registers (I <= 2048)
 constexpr long kProducerWait = 1L << 22;
@@ -70,7 +77,8 @@ constexpr long kConsumerWait = 1L << 24;
 constexpr long kEpilogueWait = 1L << 25;
 constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps
 
-enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3 };
+enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3, D_ROUTE = 4 };
+constexpr int kMaxPairs = kMaxT * 32;
 
 struct Desc {
     int type;
@@ -116,10 +124,20 @@ struct Smem {
     uint64_t* aempty;
     uint64_t* tfull;
     uint64_t* tfree;
+    uint64_t* route_bar;  // consumers -> producer: routing of the batch is ready
     int* flag;
-    int* chosen;     // [kMaxT][32]
-    int* ent;        // [kMaxT * 32] union scratch
+    int* chosen;     // [kMaxT][32] chosen experts per token, slot order
+    int* ent;        // [kMaxPairs] union scratch
     uint32_t* bmap;  // [32]
+    // routing of the batch, identical in every CTA
+    float* rt_w;     // [kMaxPairs] gate weights by (token, slot)
+    int* rt_pair_of; // [kMaxPairs] pair index by (token, slot)
+    int* rt_uniq;    // [kMaxPairs] distinct experts ascending
+    int* rt_off;     // [kMaxPairs + 1] pair offsets per distinct expert
+    int* rt_ptok;    // [kMaxPairs] token of each pair
+    int* rt_U;       // [1] number of distinct experts
+    int* bpre;       // [33] prefix popcounts of the expert bitmap
+    uint8_t* qscratch;  // [kConsumerWarps][256] Q8_0 staging (aliases the activation slots)
 };
 
 __host__ __device__ inline size_t a16(size_t v) { return (v + 15) & ~size_t(15); }
@@ -134,7 +152,9 @@ __host__ __device__ inline Layout layout_of(const FusedParams& p) {
     const int nbH = p.H / 32;
     size_t o = 0;
     L.ring = o; o += a16(slot * p.nstage);
-    L.act = o; o += a16(static_cast<size_t>(p.act_bytes) * kActSlots);
+    // the activation slots (down tiles) double as Q8_0 staging before routing
+    const size_t act = static_cast<size_t>(p.act_bytes) * kActSlots, qstage = static_cast<size_t>(kConsumerWarps) * 256;
+    L.act = o; o += a16(act > qstage ? act : qstage);
     L.xs = o; o += a16(static_cast<size_t>(p.T) * p.H * 2);
     L.qx = o; o += a16(static_cast<size_t>(p.T) * nbH * 40);
     L.bias = o; o += a16(sizeof(float) * p.E);
@@ -142,8 +162,8 @@ __host__ __device__ inline Layout layout_of(const FusedParams& p) {
     L.task = o; o += a16(sizeof(Task) * kTaskSlots);
     L.gbuf = o; o += a16(sizeof(float) * 2 * kTaskSlots * kMaxT * kUgTileRows);
     L.red = o; o += a16(sizeof(double) * kConsumerWarps * kMaxRouterRows * kMaxT);
-    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 2 * kActSlots + 2 * kTaskSlots));
-    L.misc = o; o += a16(sizeof(int) * (4 + 2 * kMaxT * 32 + 32));
+    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 2 * kActSlots + 2 * kTaskSlots + 1));
+    L.misc = o; o += a16(sizeof(int) * (4 + 2 * kMaxPairs + 32 + 5 * kMaxPairs + 2 + 33));
     L.total = o;
     return L;
 }
@@ -171,10 +191,19 @@ __device__ Smem carve(uint8_t* base, const FusedParams& p) {
     s.aempty = s.afull + kActSlots;
     s.tfull = s.aempty + kActSlots;
     s.tfree = s.tfull + kTaskSlots;
+    s.route_bar = s.tfree + kTaskSlots;
     s.flag = reinterpret_cast<int*>(base + L.misc);
     s.chosen = s.flag + 4;
-    s.ent = s.chosen + kMaxT * 32;
-    s.bmap = reinterpret_cast<uint32_t*>(s.ent + kMaxT * 32);
+    s.ent = s.chosen + kMaxPairs;
+    s.bmap = reinterpret_cast<uint32_t*>(s.ent + kMaxPairs);
+    s.rt_w = reinterpret_cast<float*>(s.bmap + 32);
+    s.rt_pair_of = reinterpret_cast<int*>(s.rt_w + kMaxPairs);
+    s.rt_uniq = s.rt_pair_of + kMaxPairs;
+    s.rt_off = s.rt_uniq + kMaxPairs;
+    s.rt_ptok = s.rt_off + kMaxPairs + 1;
+    s.rt_U = s.rt_ptok + kMaxPairs;
+    s.bpre = s.rt_U + 1;
+    s.qscratch = s.act;
     return s;
 }
 
@@ -229,9 +258,17 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
     uint32_t sphase = 0, aphase = 0;
     long n_issued = 0, n_act = 0;
     int U = -1;
-    bool ok = true;
+    bool ok = true, marked = false;
 
-    auto acquire_stage = [&]() -> bool { return mbar_wait(&s.empty[stage], sphase ^ 1u, kProducerWait); };
+    auto acquire_stage = [&]() -> bool {
+        if (n_issued >= kMaxInflight) {  // at most kMaxInflight copies in flight
+            const long older = n_issued - kMaxInflight;
+            if (!mbar_wait(&s.full[older % p.nstage], static_cast<uint32_t>((older / p.nstage) & 1),
+                           kProducerWait))
+                return false;
+        }
+        return mbar_wait(&s.empty[stage], sphase ^ 1u, kProducerWait);
+    };
     auto advance = [&]() {
         ++n_issued;
         if (++stage == p.nstage) {
@@ -263,17 +300,27 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
             ok = issue(d, p.w_router + static_cast<size_t>(d.e) * p.H, 4u * p.H * d.nrows, nullptr, 0);
             continue;
         }
+        if (!marked) {  // router rows of this CTA are all queued: the consumers route next
+            if (!acquire_stage()) {
+                ok = false;
+                break;
+            }
+            s.desc[stage].type = D_ROUTE;
+            mbar_arrive(&s.full[stage]);
+            advance();
+            marked = true;
+        }
         int t = cur - nrt;
         int kind, u, j;  // kind: 0 up/gate, 1 down; u = -1 shared
         if (hs && t < nug) {
             kind = 0; u = -1; j = t;
         } else {
             if (U < 0) {
-                if (!wait_counter_geq(&p.sync->route_ready, 1, kProducerWait)) {
+                if (!mbar_wait(s.route_bar, 0, kProducerWait)) {
                     ok = false;
                     break;
                 }
-                U = __ldcg(p.n_unique);
+                U = *reinterpret_cast<volatile int*>(s.rt_U);
             }
             t -= hs * nug;
             if (t < U * nug) {
@@ -299,11 +346,11 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                 d.pair[i] = P + i;
             }
         } else {
-            d.e = __ldcg(p.uniq + u);
-            const int p0 = __ldcg(p.offsets + u), p1 = __ldcg(p.offsets + u + 1);
+            d.e = s.rt_uniq[u];
+            const int p0 = s.rt_off[u], p1 = s.rt_off[u + 1];
             d.n_tok = p1 - p0;
             for (int i = 0; i < d.n_tok; ++i) {
-                d.tok[i] = __ldcg(p.pair_tok + p0 + i);
+                d.tok[i] = s.rt_ptok[p0 + i];
                 d.pair[i] = p0 + i;
             }
         }
@@ -357,7 +404,12 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         }
     }
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
-    // tell the consumers to stop
+    // tell the consumers to stop (after the route marker, if none was queued yet)
+    if (!marked && acquire_stage()) {
+        s.desc[stage].type = D_ROUTE;
+        mbar_arrive(&s.full[stage]);
+        advance();
+    }
     if (acquire_stage()) {
         s.desc[stage].type = D_EXIT;
         mbar_arrive(&s.full[stage]);
@@ -441,20 +493,76 @@ __device__ __forceinline__ void quantize_block_thread(const uint16_t* src, uint4
 }
 
 // ------------------------------------------------------------------ consumers
+// Q8_0 of every token's x (all consumer threads, four per 32-block), stored
+// permuted for dp4a against qtype QT.  Same arithmetic as q8_0_lane.
 template <int QT>
+__device__ void quantize_x(const FusedParams& p, const Smem& s) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int nbH = p.H / 32, ntask = p.T * nbH * 4;
+    uint8_t* scr = s.qscratch + (tid >> 5) * 256 + (lane >> 2) * 32;  // this lane group's block
+    for (int base = 0; base < ntask; base += kConsumers) {
+        const int task = base + tid;
+        const bool active = task < ntask;
+        const int blk = task >> 2, part = task & 3;
+        float v[8];
+        float amax = 0.0f;
+        if (active) {
+            const int t = blk / nbH, b = blk % nbH;
+            const uint4 u = reinterpret_cast<const uint4*>(s.xs + static_cast<size_t>(t) * p.H + 32 * b)[part];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = bf16_bits_to_f32(static_cast<uint16_t>(w[i]));
+                v[2 * i + 1] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] >> 16));
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float d = __fdiv_rn(amax, 127.0f);
+        int sum = 0;
+        uint32_t packed[2] = {0u, 0u};
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int qi = 0;
+                if (d != 0.0f) qi = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f));
+                sum += qi;
+                packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
+            }
+            *reinterpret_cast<uint2*>(scr + 8 * part) = make_uint2(packed[0], packed[1]);
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        __syncwarp();
+        if (active) {
+            uint32_t o[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int w = 2 * part + k;
+                uint32_t word = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) word |= static_cast<uint32_t>(scr[perm_src<QT>(w, i)]) << (8 * i);
+                o[k] = word;
+            }
+            uint32_t* dst = reinterpret_cast<uint32_t*>(part < 2 ? s.q0 + blk : s.q1 + blk) + 2 * (part & 1);
+            *reinterpret_cast<uint2*>(dst) = make_uint2(o[0], o[1]);
+            if (part == 0) {
+                s.qd[blk] = d;
+                s.qs[blk] = sum;
+            }
+        }
+        __syncwarp();
+    }
+}
+
 __device__ void consumer_init(const FusedParams& p, const Smem& s) {
     const int tid = threadIdx.x;
-    const int nbH = p.H / 32;
     const int n16 = p.T * p.H / 8;
     for (int i = tid; i < n16; i += kConsumers)
         reinterpret_cast<uint4*>(s.xs)[i] = reinterpret_cast<const uint4*>(p.x)[i];
     for (int e = tid; e < p.E; e += kConsumers) s.bias[e] = __ldg(p.bias + e);
-    consumers_sync();
-    for (int blk = tid; blk < p.T * nbH; blk += kConsumers) {
-        const int t = blk / nbH, b = blk % nbH;
-        quantize_block_thread<QT>(s.xs + static_cast<size_t>(t) * p.H + 32 * b, s.q0 + blk, s.q1 + blk,
-                                  s.qd + blk, s.qs + blk);
-    }
     consumers_sync();
 }
 
@@ -508,23 +616,39 @@ __device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int 
         double sum = 0.0;
         for (int w = 0; w < kConsumerWarps; ++w) sum += s.red[(w * kMaxRouterRows + q) * kMaxT + t];
         p.logits[static_cast<size_t>(t) * p.E + e0 + q] = __double2float_rn(sum);
+        red_release_add_gpu(&p.sync->router_done, 1);  // one count per logit
     }
 }
 
-// Selection and union for the whole batch, run by all consumer threads of the
-// CTA that finished the last router row.  noaux_tc (DeepSeek-V3 routing, as
-// [HN] "구현된 주요 기능" names it): s = sigmoid(logit), b = s + bias; group
-// score = sum of the two largest b; keep topk_group groups; keep the top_k
-// experts of kept groups by b; ties to the lower index.  Each kept group /
-// expert finds its rank by counting the candidates that order before it.
-__device__ void route_batch(const FusedParams& p, const Smem& s) {
+// Selection and union for the whole batch, computed by all consumer threads
+// of every CTA into shared memory once every logit has been counted.
+// noaux_tc (DeepSeek-V3 routing, as [HN] "구현된 주요 기능" names it):
+// s = sigmoid(logit), b = s + bias; group score = sum of the two largest b;
+// keep topk_group groups; keep the top_k experts of kept groups by b; ties to
+// the lower index.  A kept group / expert finds its rank by counting the
+// candidates that order before it (vectorised scans over shared memory).
+__device__ void route_cta(const FusedParams& p, const Smem& s) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = p.T, K = p.K, E = p.E, G = p.G, TG = p.TG, gsz = E / G;
-    float* sv = reinterpret_cast<float*>(s.xs);  // [T][E] unbiased scores
-    float* bv = sv + T * E;                      // [T][E] biased scores
-    float* gs = bv + T * E;                      // [T][G] group scores
-    int* gk = reinterpret_cast<int*>(gs + T * G);  // [T][G] kept
-    int* ch = s.chosen;                            // [T][32]
+    float* sv = reinterpret_cast<float*>(s.xs);    // [T][E] unbiased scores
+    float* bv = sv + T * E;                        // [T][E] biased scores
+    float* gs = bv + T * E;                        // [T][G] group scores
+    int* kg = reinterpret_cast<int*>(gs + T * G);  // [T][TG] kept groups (any order)
+    int* ch = s.chosen;                            // [T][32] chosen experts, slot order
+    int* bpre = s.bpre;
+    const bool vec = (gsz % 4 == 0) && (E % 4 == 0);
+    if (tid == 0) {
+        bool okc = false;
+        for (long i = 0; i < kConsumerWait; ++i) {
+            if (ld_relaxed_gpu(&p.sync->router_done) >= T * E) {
+                okc = ld_acquire_gpu(&p.sync->router_done) >= T * E;
+                break;
+            }
+            __nanosleep(32);
+        }
+        if (!okc) record_status(p.status, MOE_EDEVICE_TIMEOUT);
+    }
+    consumers_sync();
     for (int i = tid; i < T * E; i += kConsumers) {
         const int e = i % E;
         const double l = static_cast<double>(__ldcg(p.logits + i));
@@ -533,6 +657,7 @@ __device__ void route_batch(const FusedParams& p, const Smem& s) {
         bv[i] = __fadd_rn(sc, s.bias[e]);
     }
     for (int i = tid; i < T * 32; i += kConsumers) ch[i] = -1;
+    if (tid < 32) s.bmap[tid] = 0;
     consumers_sync();
     // group scores: one warp per (token, group); lane-local top-2, then a warp merge
     for (int pg = warp; pg < T * G; pg += kConsumerWarps) {
@@ -558,6 +683,7 @@ __device__ void route_batch(const FusedParams& p, const Smem& s) {
         if (lane == 0) gs[pg] = __fadd_rn(m1, m2);
     }
     consumers_sync();
+    // kept groups: rank each group's score among its token's groups
     for (int i = tid; i < T * G; i += kConsumers) {
         const int t = i / G, g = i % G;
         const float v = gs[i];
@@ -566,88 +692,106 @@ __device__ void route_batch(const FusedParams& p, const Smem& s) {
             const float w = gs[t * G + g2];
             r += (w > v) || (w == v && g2 < g);
         }
-        gk[i] = r < TG;
+        if (r < TG) kg[t * TG + r] = g;
     }
     consumers_sync();
+    // experts: rank each expert of a kept group among all experts of kept groups
     for (int i = tid; i < T * E; i += kConsumers) {
-        const int t = i / E, e = i % E;
-        if (!gk[t * G + e / gsz]) continue;
+        const int t = i / E, e = i % E, ge = e / gsz;
+        bool kept = false;
+        for (int j = 0; j < TG; ++j) kept |= kg[t * TG + j] == ge;
+        if (!kept) continue;
         const float v = bv[i];
         int r = 0;
-        for (int g2 = 0; g2 < G; ++g2) {
-            if (!gk[t * G + g2]) continue;
-            const float* bg = bv + t * E + g2 * gsz;
-            const int ebase = g2 * gsz;
-            for (int k = 0; k < gsz; ++k) {
-                const float w = bg[k];
-                r += (w > v) || (w == v && ebase + k < e);
+        for (int j = 0; j < TG; ++j) {
+            const int base = kg[t * TG + j] * gsz;
+            const float* bg = bv + t * E + base;
+            if (vec) {
+                const float4* bg4 = reinterpret_cast<const float4*>(bg);
+#pragma unroll 4
+                for (int q = 0; q < gsz / 4; ++q) {
+                    const float4 w = bg4[q];
+                    const int x = base + 4 * q;
+                    r += (w.x > v) | ((w.x == v) & (x < e));
+                    r += (w.y > v) | ((w.y == v) & (x + 1 < e));
+                    r += (w.z > v) | ((w.z == v) & (x + 2 < e));
+                    r += (w.w > v) | ((w.w == v) & (x + 3 < e));
+                }
+            } else {
+                for (int q = 0; q < gsz; ++q) r += (bg[q] > v) | ((bg[q] == v) & (base + q < e));
             }
         }
         if (r < K) ch[t * 32 + r] = e;
     }
     consumers_sync();
-    if (tid < T) {
-        const int t = tid;
-        float den = 0.0f;
-        for (int k = 0; k < K; ++k) {
-            int e = ch[t * 32 + k];
-            if (e < 0 || e >= E) {  // only reachable with NaN scores: keep indices in range, flag it
-                record_status(p.status, MOE_EDEVICE_INDEX);
-                e = 0;
-                ch[t * 32 + k] = 0;
-            }
-            den = __fadd_rn(den, sv[t * E + e]);
+    // per token (warp t, lane k = slot): guard, gate weight, entry, bitmap
+    if (warp < T) {
+        const int t = warp;
+        int e = lane < K ? ch[t * 32 + lane] : 0;
+        if (lane < K && (e < 0 || e >= E)) {  // only reachable with NaN scores
+            record_status(p.status, MOE_EDEVICE_INDEX);
+            e = 0;
         }
-        for (int k = 0; k < K; ++k) {
-            const int e = ch[t * 32 + k];
-            p.idx[t * K + k] = e;
-            p.w[t * K + k] = __fmul_rn(__fdiv_rn(sv[t * E + e], den), p.rsf);
+        const float sk = lane < K ? sv[t * E + e] : 0.0f;
+        float den = 0.0f;  // sum in slot order, as the definition orders it
+        for (int j = 0; j < K; ++j) den = __fadd_rn(den, __shfl_sync(0xffffffffu, sk, j));
+        if (lane < K) {
+            ch[t * 32 + lane] = e;
+            s.rt_w[t * K + lane] = __fmul_rn(__fdiv_rn(sk, den), p.rsf);
+            s.ent[t * K + lane] = e;
+            atomicOr(&s.bmap[e >> 5], 1u << (e & 31));
         }
     }
+    consumers_sync();
+    if (warp == 0) {  // exclusive prefix of the bitmap's popcounts
+        const int c = __popc(s.bmap[lane]);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n2 = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += n2;
+        }
+        bpre[lane] = incl - c;
+        if (lane == 31) bpre[32] = incl;
+    }
+    consumers_sync();
     // union of the T*K entries: (expert ascending, token ascending) positions
     const int n = T * K;
-    if (tid < 32) s.bmap[tid] = 0;
-    consumers_sync();
     for (int i = tid; i < n; i += kConsumers) {
-        const int e = ch[(i / K) * 32 + (i % K)];
-        s.ent[i] = e;
-        atomicOr(&s.bmap[e >> 5], 1u << (e & 31));
-    }
-    consumers_sync();
-    for (int i = tid; i < n; i += kConsumers) {
-        const int t = i / K, k = i % K, e = s.ent[i];
+        const int t = i / K, e = s.ent[i];
         int before = 0, same_before = 0, first = 1;
         for (int jx = 0, tj = 0, kj = 0; jx < n; ++jx) {  // tj = jx / K without a division
             const int ej = s.ent[jx];
             before += ej < e;
-            same_before += (ej == e) && (tj < t);
-            if (ej == e && jx < i) first = 0;
+            same_before += (ej == e) & (tj < t);
+            first &= !((ej == e) & (jx < i));
             if (++kj == K) {
                 kj = 0;
                 ++tj;
             }
         }
-        int rank = __popc(s.bmap[e >> 5] & ((1u << (e & 31)) - 1u));
-        for (int wd = 0; wd < (e >> 5); ++wd) rank += __popc(s.bmap[wd]);
+        const int rank = bpre[e >> 5] + __popc(s.bmap[e >> 5] & ((1u << (e & 31)) - 1u));
         const int pos = before + same_before;
-        p.pair_tok[pos] = t;
-        p.pair_slot[pos] = k;
-        p.pair_of[i] = pos;
+        s.rt_ptok[pos] = t;
+        s.rt_pair_of[i] = pos;
         if (first) {
-            p.uniq[rank] = e;
-            p.offsets[rank] = before;
+            s.rt_uniq[rank] = e;
+            s.rt_off[rank] = before;
         }
     }
     if (tid == 0) {
-        int U = 0;
-        for (int wd = 0; wd < 32; ++wd) U += __popc(s.bmap[wd]);
-        *p.n_unique = U;
-        p.offsets[U] = n;
+        const int U = bpre[32];
+        *s.rt_U = U;
+        s.rt_off[U] = n;
     }
     consumers_sync();
-    if (tid == 0) {
-        __threadfence();
-        st_release_gpu(&p.sync->route_ready, 1);
+    if (tid == 0) mbar_arrive(s.route_bar);
+    // the routing outputs the caller can see, written once (off the critical path)
+    if (blockIdx.x == 0) {
+        for (int i = tid; i < n; i += kConsumers) {
+            p.idx[i] = ch[(i / K) * 32 + (i % K)];
+            p.w[i] = s.rt_w[i];
+        }
     }
 }
 
@@ -824,7 +968,7 @@ template <int QT, int NT>
 __device__ void consumer(const FusedParams& p, const Smem& s) {
     const int tid = threadIdx.x, lane = tid & 31;
     const size_t slot_bytes = static_cast<size_t>(p.stage_bytes) + kScaleBytes;
-    consumer_init<QT>(p, s);
+    consumer_init(p, s);
     int stage = 0, aslot = 0, tb = 0;
     uint32_t phase = 0, aphase = 0;
     uint32_t tph[kTaskSlots] = {0, 0};
@@ -857,20 +1001,18 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
         tb ^= 1;
     };
     int type = next_type();
-    // phase A: router rows
+    // phase A: router rows, then (at the route marker) Q8_0 of x and the routing
     while (type == D_ROUTER) {
         const int e0 = s.desc[stage].e, nrows = s.desc[stage].nrows;
         consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes);
         release();
-        consumers_sync();
-        if (tid == 0) {
-            __threadfence();
-            const bool last = atomicAdd(&p.sync->router_done, nrows) + nrows == p.E;
-            if (last) __threadfence();
-            s.flag[0] = last;
-        }
-        consumers_sync();
-        if (s.flag[0]) route_batch(p, s);
+        type = next_type();
+    }
+    quantize_x<QT>(p, s);
+    consumers_sync();
+    if (type == D_ROUTE) {
+        route_cta(p, s);
+        release();
         type = next_type();
     }
     // phase B: up/gate tiles
@@ -1006,8 +1148,8 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s) {
                     const int t = i / nr, c = c0 + i % nr;
                     float o = p.has_shared ? __ldcg(p.y + static_cast<size_t>(P + t) * p.H + c) : 0.0f;
                     for (int k = 0; k < p.K; ++k) {
-                        const int pr = __ldcg(p.pair_of + t * p.K + k);
-                        const float wk = __ldcg(p.w + t * p.K + k);
+                        const int pr = s.rt_pair_of[t * p.K + k];
+                        const float wk = s.rt_w[t * p.K + k];
                         o = __fadd_rn(o, __fmul_rn(wk, __ldcg(p.y + static_cast<size_t>(pr) * p.H + c)));
                     }
                     if (p.out_bf16) {
@@ -1030,6 +1172,15 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const Smem s = carve(smem_raw, p);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Touch every parameter word now, while the memory system is idle: a
+    // constant-cache miss on a parameter first read in the middle of the
+    // kernel would queue behind the weight stream.
+    {
+        const int* pw = reinterpret_cast<const int*>(&p);
+        int acc = 0;
+        for (int i = lane; i < static_cast<int>(sizeof(FusedParams) / 4); i += 32) acc ^= pw[i];
+        if (acc == 0x7fffffff && tid == kThreadsF) s.flag[3] = acc;  // keeps the reads
+    }
     if (tid == 0) {
         for (int i = 0; i < p.nstage; ++i) {
             mbar_init(&s.full[i], 1);
@@ -1043,6 +1194,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfull[i], kConsumerWarps);
             mbar_init(&s.tfree[i], 1);
         }
+        mbar_init(s.route_bar, 1);
         fence_mbar_init();
     }
     __syncthreads();

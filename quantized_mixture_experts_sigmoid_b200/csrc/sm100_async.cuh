@@ -98,10 +98,28 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Polls *p (acquire, gpu scope) until it reaches `target`; false after `limit` polls.
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Fire-and-forget add with release semantics (orders this thread's earlier writes before it).
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Polls *p until it reaches `target`, then orders later loads after it
+// (relaxed polls and one fence: an acquire load per poll would invalidate the
+// SM's L1 every time); false after `limit` polls.
 __device__ __forceinline__ bool wait_counter_geq(const int* p, int target, long limit) {
     for (long i = 0; i < limit; ++i) {
-        if (ld_acquire_gpu(p) >= target) return true;
+        if (ld_relaxed_gpu(p) >= target) {
+            fence_acquire_gpu();
+            return true;
+        }
         __nanosleep(i < 64 ? 32 : 256);
     }
     return false;
