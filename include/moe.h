@@ -24,6 +24,10 @@
  *  - bf16 values are passed as their 16-bit patterns (uint16_t).
  *  - Not thread-safe per workspace: two calls in flight that share a `ws`
  *    race on it.
+ *  - The first 16 KiB of every workspace belong to the library: a status
+ *    word, and for moe_layer_forward counters, router score slots and a
+ *    launch counter that persist from one call to the next.  Zero-fill a
+ *    workspace once before its first use and do not write into it afterwards.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -243,7 +247,9 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
 /*
  * Read (and clear when `clear` != 0) the device status word that kernels of
  * moe_layer_forward / moe_expert_ffn_q record in `ws`.  Synchronises `stream`.
- * *status receives MOE_OK or the first device-side MOE_E* code.
+ * *status receives MOE_OK or the first device-side MOE_E* code.  A clear also
+ * zeroes the layer's counters (needed after a device-side timeout, which can
+ * leave them mid-count); the launch counter is kept.
  */
 int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream);
 

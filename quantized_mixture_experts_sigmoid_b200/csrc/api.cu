@@ -178,7 +178,8 @@ bool fused_params(FusedParams& f, const LayerWs& L, void* ws, const uint16_t* x,
     f.sync = reinterpret_cast<FusedSync*>(base + kWsSyncOff);
     f.ug_done = reinterpret_cast<int32_t*>(base + kWsUgDoneOff);
     f.rb_done = reinterpret_cast<int32_t*>(base + kWsRbDoneOff);
-    f.logits = L.logits;
+    f.epoch = reinterpret_cast<uint32_t*>(base + kWsEpochOff);
+    f.scores = reinterpret_cast<unsigned long long*>(base + kWsScoresOff);
     f.n_unique = L.n_unique;
     f.uniq = L.uniq;
     f.offsets = L.offsets;
@@ -416,7 +417,8 @@ int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream) 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int32_t h = 0;
     if (cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ECUDA;
-    if (clear && cudaMemsetAsync(ws, 0, kWsHeader, st) != cudaSuccess) return MOE_ECUDA;
+    // the launch counter at the end of the header survives a clear
+    if (clear && cudaMemsetAsync(ws, 0, kWsEpochOff, st) != cudaSuccess) return MOE_ECUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ECUDA;
     *status = h;
     return MOE_OK;

@@ -17,9 +17,10 @@ namespace moe {
 constexpr int kWarp = 32;
 constexpr int kQBlock = 32;  // Q8_0 block length
 
-// Every workspace starts with a control header: the device status word at
-// offset 0, then the fused kernel's self-resetting counters.
-constexpr size_t kWsHeader = 8192;
+// Every workspace starts with a control header owned by the library: the
+// device status word at offset 0, then the fused kernel's self-resetting
+// counters, its router score slots and its launch counter.
+constexpr size_t kWsHeader = 16384;
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
     return __uint_as_float(static_cast<uint32_t>(b) << 16);

@@ -8,32 +8,37 @@
 // weight stream from HBM (176.5 MB per decode token for GLM-5.2's shape), so
 // the design goal is to keep HBM busy from the first byte to the last.
 //
-// Roles (one CTA per SM):
-//  * warp 17, the producer, streams weight rows into a shared-memory ring
+// Roles (one CTA per SM, 20 warps):
+//  * warp 18, the producer, streams weight rows into a shared-memory ring
 //    with bulk copies (cp.async.bulk, non-multicast TMA) completing on
 //    mbarriers;
 //  * warps 0-15, the consumers, take one ring stage at a time and form the
 //    integer dot products with dp4a;
-//  * warp 16, the epilogue warp, finishes tiles handed over through a
-//    double-buffered mbarrier queue (SwiGLU and Q8_0 of h for up/gate tiles;
+//  * warps 16-17, the epilogue warps, each finish the tiles handed over
+//    through one task slot (SwiGLU and Q8_0 of h for up/gate tiles;
 //    completion counting and the combine for down tiles), so the consumers
-//    never wait on fences or atomics.
+//    never wait on fences or atomics;
+//  * warp 19, the helper, first routes the batch (every CTA computes the same
+//    routing from the published router scores, in registers), then copies
+//    each down tile's activation records once the expert's h is complete, so
+//    the producer never waits on another CTA.
 //
 // Work is one global ticket sequence claimed by the producers:
-//      router rows | shared up/gate tiles | routed up/gate tiles |
-//      shared down tiles | routed down tiles
-// so every dependency points to an earlier ticket and every CTA sees its
-// stages in that order.  After its last router row a producer queues a
-// zero-byte route marker; at the marker the consumers wait until every logit
-// of the batch has been counted, then compute the noaux_tc selection and the
-// batch union themselves (all consumer threads, rank-based, in shared memory:
-// every CTA reaches the same result) and hand it to their producer through an
-// mbarrier.  Routing therefore costs one global round trip (the logit count)
-// rather than a publish by one CTA and a read-back by all.  An up/gate tile is 32 rows of h for one expert; its epilogue
-// writes Q8_0(h) as a pre-permuted activation record.  A down tile waits for
-// its expert's h tiles, then copies the records of its pairs next to its
-// weight stages.  The CTA that completes a row block of the output combines
-// it (shared + sum_k w_k y_k in slot order), so the result is deterministic.
+//      router rows | shared up/gate tiles | then, per distinct routed expert
+//      u: its up/gate tiles, followed by the down tiles of expert u - 3; the
+//      last routed experts' down tiles at the end, the shared expert's down
+//      tiles before the very last expert's,
+// so every dependency points to an earlier ticket, far enough back that it is
+// usually complete when claimed.  The consumers that finish a router row
+// publish its scores (sigmoid of the fp32-rounded logit) in 64-bit slots
+// tagged with the launch number; the helper warps poll those slots, so the
+// data and its readiness arrive in one load.  A producer claims routed tiles
+// once its helper warp has routed.  An up/gate tile is 32 rows of h for one
+// expert; its epilogue writes Q8_0(h) as a pre-permuted activation record.  A
+// down tile's weight stages stream at once; its records follow when the
+// expert's h tiles are all done.  The CTA that completes a row block of the
+// output combines it (shared + sum_k w_k y_k in slot order), so the result is
+// deterministic.
 //
 // NT is the compile-time token capacity: NT = 1 keeps the token's activations
 // in registers; NT = 4 reads them from shared memory.
@@ -54,9 +59,11 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kEpilogueWarp = kConsumerWarps;
-constexpr int kProducerWarp = kConsumerWarps + 1;
-constexpr int kThreadsF = (kConsumerWarps + 2) * 32;
+constexpr int kEpilogueWarps = 2;    // one per task slot
+constexpr int kEpilogueWarp0 = kConsumerWarps;
+constexpr int kProducerWarp = kEpilogueWarp0 + kEpilogueWarps;
+constexpr int kHelperWarp = kProducerWarp + 1;  // routing, then the activation copies
+constexpr int kThreadsF = (kHelperWarp + 1) * 32;
 constexpr int kMaxT = kFusedMaxTokens;
 constexpr int kStageRows = 16;       // up/gate rows per stage (one per consumer warp)
 constexpr int kUgTileRows = 32;      // one Q8_0 block of h
@@ -64,7 +71,7 @@ constexpr int kDownStagesPerTile = 2;
 constexpr int kMaxRouterRows = 4;    // router rows per stage
 constexpr int kMaxDownRowsPerWarp = 4;
 constexpr int kActSlots = 2;
-constexpr int kTaskSlots = 2;
+constexpr int kTaskSlots = kEpilogueWarps;
 constexpr int kScaleBytes = 256;     // room after each stage for its rows' fp32 scales
 // Copies a producer keeps in flight.  Enough to cover HBM latency at full
 // bandwidth; more only lengthens the memory queues, and every other request
@@ -76,8 +83,10 @@ constexpr long kProducerWait = 1L << 22;
 constexpr long kConsumerWait = 1L << 24;
 constexpr long kEpilogueWait = 1L << 25;
 constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps
+constexpr int kDownLag = 8;          // routed experts between an expert's up/gate and down tiles
+constexpr int kMaxExpertsPerLane = 8; // warp routing: E <= 32 * 8
 
-enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3, D_ROUTE = 4 };
+enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3 };
 constexpr int kMaxPairs = kMaxT * 32;
 
 struct Desc {
@@ -97,7 +106,18 @@ struct Desc {
     int pair[kMaxT];
 };
 
-// A finished tile handed to the epilogue warp.
+// A down tile's activation-record copy, posted by the producer and issued by
+// the helper warp once the expert's h is complete.
+struct ActReq {
+    const uint8_t* src;
+    uint32_t bytes;
+    int cslot;
+    int need;   // h tiles the expert must have finished
+    int exit;
+    int pad[2];
+};
+
+// A finished tile handed to an epilogue warp.
 struct Task {
     int type;  // D_UG, D_DOWN or D_EXIT
     int n_tok, blk, cslot, n_experts;
@@ -124,11 +144,12 @@ struct Smem {
     uint64_t* aempty;
     uint64_t* tfull;
     uint64_t* tfree;
-    uint64_t* route_bar;  // consumers -> producer: routing of the batch is ready
+    uint64_t* route_bar;  // helper warp -> producer: routing of the batch is ready
+    uint64_t* areq_full;  // [kActSlots] producer -> helper: request posted
+    uint64_t* areq_free;  // [kActSlots] helper -> producer: request taken
+    ActReq* areq;         // [kActSlots]
     int* flag;
-    int* chosen;     // [kMaxT][32] chosen experts per token, slot order
-    int* ent;        // [kMaxPairs] union scratch
-    uint32_t* bmap;  // [32]
+    uint32_t* tag;   // [1] this launch's score tag
     // routing of the batch, identical in every CTA
     float* rt_w;     // [kMaxPairs] gate weights by (token, slot)
     int* rt_pair_of; // [kMaxPairs] pair index by (token, slot)
@@ -136,14 +157,12 @@ struct Smem {
     int* rt_off;     // [kMaxPairs + 1] pair offsets per distinct expert
     int* rt_ptok;    // [kMaxPairs] token of each pair
     int* rt_U;       // [1] number of distinct experts
-    int* bpre;       // [33] prefix popcounts of the expert bitmap
-    uint8_t* qscratch;  // [kConsumerWarps][256] Q8_0 staging (aliases the activation slots)
 };
 
 __host__ __device__ inline size_t a16(size_t v) { return (v + 15) & ~size_t(15); }
 
 struct Layout {
-    size_t ring, act, xs, qx, bias, desc, task, gbuf, red, bars, misc, total;
+    size_t ring, act, xs, qx, bias, desc, task, areq, gbuf, red, bars, misc, total;
 };
 
 __host__ __device__ inline Layout layout_of(const FusedParams& p) {
@@ -152,18 +171,17 @@ __host__ __device__ inline Layout layout_of(const FusedParams& p) {
     const int nbH = p.H / 32;
     size_t o = 0;
     L.ring = o; o += a16(slot * p.nstage);
-    // the activation slots (down tiles) double as Q8_0 staging before routing
-    const size_t act = static_cast<size_t>(p.act_bytes) * kActSlots, qstage = static_cast<size_t>(kConsumerWarps) * 256;
-    L.act = o; o += a16(act > qstage ? act : qstage);
+    L.act = o; o += a16(static_cast<size_t>(p.act_bytes) * kActSlots);
     L.xs = o; o += a16(static_cast<size_t>(p.T) * p.H * 2);
     L.qx = o; o += a16(static_cast<size_t>(p.T) * nbH * 40);
     L.bias = o; o += a16(sizeof(float) * p.E);
     L.desc = o; o += a16(sizeof(Desc) * p.nstage);
     L.task = o; o += a16(sizeof(Task) * kTaskSlots);
+    L.areq = o; o += a16(sizeof(ActReq) * kActSlots);
     L.gbuf = o; o += a16(sizeof(float) * 2 * kTaskSlots * kMaxT * kUgTileRows);
     L.red = o; o += a16(sizeof(double) * kConsumerWarps * kMaxRouterRows * kMaxT);
-    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 2 * kActSlots + 2 * kTaskSlots + 1));
-    L.misc = o; o += a16(sizeof(int) * (4 + 2 * kMaxPairs + 32 + 5 * kMaxPairs + 2 + 33));
+    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 4 * kActSlots + 2 * kTaskSlots + 1));
+    L.misc = o; o += a16(sizeof(int) * (4 + 4 + 5 * kMaxPairs + 2));
     L.total = o;
     return L;
 }
@@ -182,6 +200,7 @@ __device__ Smem carve(uint8_t* base, const FusedParams& p) {
     s.bias = reinterpret_cast<float*>(base + L.bias);
     s.desc = reinterpret_cast<Desc*>(base + L.desc);
     s.task = reinterpret_cast<Task*>(base + L.task);
+    s.areq = reinterpret_cast<ActReq*>(base + L.areq);
     s.gbuf = reinterpret_cast<float*>(base + L.gbuf);
     s.ubuf = s.gbuf + kTaskSlots * kMaxT * kUgTileRows;
     s.red = reinterpret_cast<double*>(base + L.red);
@@ -192,18 +211,16 @@ __device__ Smem carve(uint8_t* base, const FusedParams& p) {
     s.tfull = s.aempty + kActSlots;
     s.tfree = s.tfull + kTaskSlots;
     s.route_bar = s.tfree + kTaskSlots;
+    s.areq_full = s.route_bar + 1;
+    s.areq_free = s.areq_full + kActSlots;
     s.flag = reinterpret_cast<int*>(base + L.misc);
-    s.chosen = s.flag + 4;
-    s.ent = s.chosen + kMaxPairs;
-    s.bmap = reinterpret_cast<uint32_t*>(s.ent + kMaxPairs);
-    s.rt_w = reinterpret_cast<float*>(s.bmap + 32);
+    s.tag = reinterpret_cast<uint32_t*>(s.flag + 4);
+    s.rt_w = reinterpret_cast<float*>(s.tag + 4);
     s.rt_pair_of = reinterpret_cast<int*>(s.rt_w + kMaxPairs);
     s.rt_uniq = s.rt_pair_of + kMaxPairs;
     s.rt_off = s.rt_uniq + kMaxPairs;
     s.rt_ptok = s.rt_off + kMaxPairs + 1;
     s.rt_U = s.rt_ptok + kMaxPairs;
-    s.bpre = s.rt_U + 1;
-    s.qscratch = s.act;
     return s;
 }
 
@@ -246,6 +263,42 @@ __device__ __forceinline__ uint32_t perm_word(int q, int lane) {
     return word;
 }
 
+// Post-routing tile order: per routed expert r its up/gate tiles, followed by
+// the down tiles of expert r - kDownLag; then the remaining routed experts'
+// down tiles, with the shared expert's (whose h was finished first) placed
+// before the last one to give that expert's h the most time.
+struct Segments {
+    int begin = 0, size = 0, kind = 0, u = 0;
+    int r = 0, phase = 0, tail = -1, shared_left = 1;
+    // Advances to the next non-empty segment; false when none is left.
+    __device__ bool next(int U, int hs, int nug, int nd) {
+        while (tail < 0) {
+            if (phase == 0) {
+                phase = 1;
+                return set(0, r, nug);
+            }
+            phase = 0;
+            const int rr = r++;
+            if (r == U) tail = U > kDownLag ? U - kDownLag : 0;
+            if (rr >= kDownLag) return set(1, rr - kDownLag, nd);
+        }
+        if (tail < U - 1) return set(1, tail++, nd);
+        if (hs && shared_left) {
+            shared_left = 0;
+            return set(1, -1, nd);
+        }
+        if (tail == U - 1) return set(1, tail++, nd);
+        size = 0;
+        return false;
+    }
+    __device__ bool set(int k, int uu, int n) {
+        kind = k;
+        u = uu;
+        size = n;
+        return true;
+    }
+};
+
 // ------------------------------------------------------------------ producer
 template <int QT>
 __device__ void producer(const FusedParams& p, const Smem& s) {
@@ -256,9 +309,10 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
     const size_t rb_ug = static_cast<size_t>(p.H) * QT / 8, rb_d = static_cast<size_t>(p.I) * QT / 8;
     int stage = 0, aslot = 0;
     uint32_t sphase = 0, aphase = 0;
-    long n_issued = 0, n_act = 0;
+    long n_issued = 0;
     int U = -1;
-    bool ok = true, marked = false;
+    bool ok = true;
+    Segments seg;
 
     auto acquire_stage = [&]() -> bool {
         if (n_issued >= kMaxInflight) {  // at most kMaxInflight copies in flight
@@ -288,10 +342,12 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         return true;
     };
 
-    int next = atomicAdd(&p.sync->ticket, 1);
+    // the first ticket of CTA b is b (no round trip before the first copy);
+    // later ones come from the shared counter
+    int next = blockIdx.x;
     while (ok) {
         const int cur = next;
-        next = atomicAdd(&p.sync->ticket, 1);
+        next = static_cast<int>(gridDim.x) + atomicAdd(&p.sync->ticket, 1);
         Desc d{};
         if (cur < nrt) {  // router rows e0 .. e0 + n - 1
             d.type = D_ROUTER;
@@ -299,16 +355,6 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
             d.nrows = min(p.rps, p.E - d.e);
             ok = issue(d, p.w_router + static_cast<size_t>(d.e) * p.H, 4u * p.H * d.nrows, nullptr, 0);
             continue;
-        }
-        if (!marked) {  // router rows of this CTA are all queued: the consumers route next
-            if (!acquire_stage()) {
-                ok = false;
-                break;
-            }
-            s.desc[stage].type = D_ROUTE;
-            mbar_arrive(&s.full[stage]);
-            advance();
-            marked = true;
         }
         int t = cur - nrt;
         int kind, u, j;  // kind: 0 up/gate, 1 down; u = -1 shared
@@ -323,18 +369,13 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                 U = *reinterpret_cast<volatile int*>(s.rt_U);
             }
             t -= hs * nug;
-            if (t < U * nug) {
-                kind = 0; u = t / nug; j = t % nug;
-            } else {
-                t -= U * nug;
-                if (hs && t < nd) {
-                    kind = 1; u = -1; j = t;
-                } else {
-                    t -= hs * nd;
-                    if (t >= U * nd) break;  // no work left
-                    kind = 1; u = t / nd; j = t % nd;
-                }
+            // walk the segment sequence forward to the segment holding ticket t
+            while (t >= seg.begin + seg.size) {
+                seg.begin += seg.size;
+                if (!seg.next(U, hs, nug, nd)) break;
             }
+            if (t >= seg.begin + seg.size) break;  // no work left
+            kind = seg.kind; u = seg.u; j = t - seg.begin;
         }
         d.cslot = u < 0 ? 0 : 1 + u;
         d.n_experts = U + hs;
@@ -372,20 +413,22 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                                kStageRows * 4);
                 }
             }
-        } else {  // down tile: rows j*dr .. j*dr+dr-1, after the expert's h is complete
+        } else {  // down tile: rows j*dr .. j*dr+dr-1; the helper warp copies its
+                  // activation records once the expert's h is complete, so the
+                  // weight stages stream meanwhile
             d.type = D_DOWN;
             d.mat = 2;
-            if (!mbar_wait(&s.aempty[aslot], aphase ^ 1u, kProducerWait) ||
-                !wait_counter_geq(p.ug_done + d.cslot, nug, kProducerWait)) {
+            if (!mbar_wait(&s.areq_free[aslot], aphase ^ 1u, kProducerWait)) {
                 ok = false;
                 break;
             }
-            fence_proxy_async_global();
-            const uint32_t abytes = static_cast<uint32_t>(d.n_tok) * p.rec_bytes;
-            mbar_arrive_expect_tx(&s.afull[aslot], abytes);
-            bulk_g2s(s.act + static_cast<size_t>(aslot) * p.act_bytes,
-                     p.qrec + static_cast<size_t>(d.pair[0]) * p.rec_bytes, abytes, &s.afull[aslot]);
-            ++n_act;
+            ActReq& rq = s.areq[aslot];
+            rq.src = p.qrec + static_cast<size_t>(d.pair[0]) * p.rec_bytes;
+            rq.bytes = static_cast<uint32_t>(d.n_tok) * p.rec_bytes;
+            rq.cslot = d.cslot;
+            rq.need = nug;
+            rq.exit = 0;
+            mbar_arrive(&s.areq_full[aslot]);
             d.aslot = aslot;
             const int c_end = min(p.H, (j + 1) * p.dr);
             for (int c0 = j * p.dr; c0 < c_end && ok; c0 += p.sr_down) {
@@ -404,11 +447,10 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         }
     }
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
-    // tell the consumers to stop (after the route marker, if none was queued yet)
-    if (!marked && acquire_stage()) {
-        s.desc[stage].type = D_ROUTE;
-        mbar_arrive(&s.full[stage]);
-        advance();
+    // tell the helper warp and the consumers to stop
+    if (mbar_wait(&s.areq_free[aslot], aphase ^ 1u, kProducerWait)) {
+        s.areq[aslot].exit = 1;
+        mbar_arrive(&s.areq_full[aslot]);
     }
     if (acquire_stage()) {
         s.desc[stage].type = D_EXIT;
@@ -420,11 +462,8 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         const long uses = n_issued / p.nstage + (st < n_issued % p.nstage ? 1 : 0);
         if (uses > 0) mbar_wait(&s.full[st], static_cast<uint32_t>((uses - 1) & 1), kProducerWait);
     }
-    for (int a = 0; a < kActSlots; ++a) {
-        const long uses = n_act / kActSlots + (a < n_act % kActSlots ? 1 : 0);
-        if (uses > 0) mbar_wait(&s.afull[a], static_cast<uint32_t>((uses - 1) & 1), kProducerWait);
-    }
 }
+
 
 // ------------------------------------------------------------------ Q8_0 helpers
 // Warp-collective: quantises one 32-value block held one value per lane to
@@ -449,111 +488,75 @@ __device__ __forceinline__ void store_q8_block_warp(float v, uint32_t* w_lo, uin
     }
 }
 
-// One thread: Q8_0 of 32 bf16 values (same arithmetic as q8_0_lane), stored
-// permuted for dp4a.
-template <int QT>
-__device__ __forceinline__ void quantize_block_thread(const uint16_t* src, uint4* q0, uint4* q1, float* qd,
-                                                      int32_t* qs) {
-    float v[32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint4 u = reinterpret_cast<const uint4*>(src)[c];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[8 * c + 2 * i] = bf16_bits_to_f32(static_cast<uint16_t>(w[i]));
-            v[8 * c + 2 * i + 1] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] >> 16));
-        }
-    }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    const float d = __fdiv_rn(amax, 127.0f);
-    int q[32];
-    int sum = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        int qi = 0;
-        if (d != 0.0f) qi = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f));
-        q[i] = qi;
-        sum += qi;
-    }
-    uint32_t o[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) word |= (static_cast<uint32_t>(q[perm_src<QT>(w, i)]) & 0xFFu) << (8 * i);
-        o[w] = word;
-    }
-    *q0 = make_uint4(o[0], o[1], o[2], o[3]);
-    *q1 = make_uint4(o[4], o[5], o[6], o[7]);
-    *qd = d;
-    *qs = sum;
-}
-
 // ------------------------------------------------------------------ consumers
-// Q8_0 of every token's x (all consumer threads, four per 32-block), stored
-// permuted for dp4a against qtype QT.  Same arithmetic as q8_0_lane.
+// Q8_0 of every token's x (all consumer threads; TPB threads per 32-block),
+// stored permuted for dp4a against qtype QT.  Same arithmetic as q8_0_lane.
+// Each thread's permuted words hold only its own elements, so no exchange
+// through shared memory is needed: thread `part` of a block owns elements
+// [part EPT, part EPT + EPT) and words [part WPT, part WPT + WPT).
 template <int QT>
-__device__ void quantize_x(const FusedParams& p, const Smem& s) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int nbH = p.H / 32, ntask = p.T * nbH * 4;
-    uint8_t* scr = s.qscratch + (tid >> 5) * 256 + (lane >> 2) * 32;  // this lane group's block
+__device__ __forceinline__ void quantize_x(const FusedParams& p, const Smem& s) {
+    constexpr int TPB = QT == 2 ? 2 : 4, EPT = 32 / TPB, WPT = 8 / TPB;
+    const int tid = threadIdx.x;
+    const int nbH = p.H / 32, ntask = p.T * nbH * TPB;
     for (int base = 0; base < ntask; base += kConsumers) {
         const int task = base + tid;
         const bool active = task < ntask;
-        const int blk = task >> 2, part = task & 3;
-        float v[8];
+        const int blk = task / TPB, part = task % TPB;
+        float v[EPT];
         float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) v[i] = 0.0f;
         if (active) {
             const int t = blk / nbH, b = blk % nbH;
-            const uint4 u = reinterpret_cast<const uint4*>(s.xs + static_cast<size_t>(t) * p.H + 32 * b)[part];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            const uint4* src = reinterpret_cast<const uint4*>(s.xs + static_cast<size_t>(t) * p.H + 32 * b + EPT * part);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                v[2 * i] = bf16_bits_to_f32(static_cast<uint16_t>(w[i]));
-                v[2 * i + 1] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] >> 16));
+            for (int c = 0; c < EPT / 8; ++c) {
+                const uint4 u = src[c];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    v[8 * c + 2 * i] = bf16_bits_to_f32(static_cast<uint16_t>(w[i]));
+                    v[8 * c + 2 * i + 1] = bf16_bits_to_f32(static_cast<uint16_t>(w[i] >> 16));
+                }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            for (int i = 0; i < EPT; ++i) amax = fmaxf(amax, fabsf(v[i]));
         }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+#pragma unroll
+        for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float d = __fdiv_rn(amax, 127.0f);
+        int q[EPT];
         int sum = 0;
-        uint32_t packed[2] = {0u, 0u};
-        if (active) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                int qi = 0;
-                if (d != 0.0f) qi = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f));
-                sum += qi;
-                packed[i >> 2] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * (i & 3));
-            }
-            *reinterpret_cast<uint2*>(scr + 8 * part) = make_uint2(packed[0], packed[1]);
+        for (int i = 0; i < EPT; ++i) {
+            int qi = 0;
+            if (d != 0.0f) qi = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f));
+            q[i] = qi;
+            sum += qi;
         }
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        __syncwarp();
-        if (active) {
-            uint32_t o[2];
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int w = 2 * part + k;
+        for (int o = 1; o < TPB; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (active) {
+            uint32_t o[WPT];
+#pragma unroll
+            for (int k = 0; k < WPT; ++k) {
                 uint32_t word = 0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) word |= static_cast<uint32_t>(scr[perm_src<QT>(w, i)]) << (8 * i);
+                for (int i = 0; i < 4; ++i) word |= (static_cast<uint32_t>(q[perm_src<QT>(k, i)]) & 0xFFu) << (8 * i);
                 o[k] = word;
             }
-            uint32_t* dst = reinterpret_cast<uint32_t*>(part < 2 ? s.q0 + blk : s.q1 + blk) + 2 * (part & 1);
-            *reinterpret_cast<uint2*>(dst) = make_uint2(o[0], o[1]);
+            if constexpr (TPB == 4) {
+                uint32_t* dst = reinterpret_cast<uint32_t*>(part < 2 ? s.q0 + blk : s.q1 + blk) + 2 * (part & 1);
+                *reinterpret_cast<uint2*>(dst) = make_uint2(o[0], o[1]);
+            } else {
+                (part == 0 ? s.q0 : s.q1)[blk] = make_uint4(o[0], o[1], o[2], o[3]);
+            }
             if (part == 0) {
                 s.qd[blk] = d;
                 s.qs[blk] = sum;
             }
         }
-        __syncwarp();
     }
 }
 
@@ -612,11 +615,15 @@ __device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int 
         }
     consumers_sync();
     if (tid < nrows * p.T) {
+        // logit rounded once to fp32, sigmoid in fp64 rounded once; published
+        // with this launch's tag in the same 64-bit word
         const int q = tid / p.T, t = tid % p.T;
         double sum = 0.0;
         for (int w = 0; w < kConsumerWarps; ++w) sum += s.red[(w * kMaxRouterRows + q) * kMaxT + t];
-        p.logits[static_cast<size_t>(t) * p.E + e0 + q] = __double2float_rn(sum);
-        red_release_add_gpu(&p.sync->router_done, 1);  // one count per logit
+        const double l = static_cast<double>(__double2float_rn(sum));
+        const float sc = __double2float_rn(1.0 / (1.0 + exp(-l)));
+        st_relaxed_gpu_u64(p.scores + static_cast<size_t>(t) * p.E + e0 + q,
+                           (static_cast<unsigned long long>(*s.tag) << 32) | __float_as_uint(sc));
     }
 }
 
@@ -627,172 +634,209 @@ __device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int 
 // keep topk_group groups; keep the top_k experts of kept groups by b; ties to
 // the lower index.  A kept group / expert finds its rank by counting the
 // candidates that order before it (vectorised scans over shared memory).
-__device__ void route_cta(const FusedParams& p, const Smem& s) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int T = p.T, K = p.K, E = p.E, G = p.G, TG = p.TG, gsz = E / G;
-    float* sv = reinterpret_cast<float*>(s.xs);    // [T][E] unbiased scores
-    float* bv = sv + T * E;                        // [T][E] biased scores
-    float* gs = bv + T * E;                        // [T][G] group scores
-    int* kg = reinterpret_cast<int*>(gs + T * G);  // [T][TG] kept groups (any order)
-    int* ch = s.chosen;                            // [T][32] chosen experts, slot order
-    int* bpre = s.bpre;
-    const bool vec = (gsz % 4 == 0) && (E % 4 == 0);
-    if (tid == 0) {
-        bool okc = false;
-        for (long i = 0; i < kConsumerWait; ++i) {
-            if (ld_relaxed_gpu(&p.sync->router_done) >= T * E) {
-                okc = ld_acquire_gpu(&p.sync->router_done) >= T * E;
-                break;
+// Order-preserving map of fp32 values to unsigned keys (+0 and -0 equal; the
+// key 0 is below every value and marks an excluded expert).
+__device__ __forceinline__ uint32_t order_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if ((b << 1) == 0) b = 0;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Compare-exchange of two (key, expert, score) candidates so that the first
+// is the better one: larger key, then lower expert index.
+__device__ __forceinline__ void cand_order(uint32_t& ka, int& ea, float& sa, uint32_t& kb, int& eb, float& sb) {
+    const bool swap = kb > ka || (kb == ka && eb < ea);
+    const uint32_t k = swap ? kb : ka;
+    const int e = swap ? eb : ea;
+    const float v = swap ? sb : sa;
+    kb = swap ? ka : kb;
+    eb = swap ? ea : eb;
+    sb = swap ? sa : sb;
+    ka = k;
+    ea = e;
+    sa = v;
+}
+
+// noaux_tc routing and the batch union of the whole batch by one warp, with
+// each lane holding experts lane + 32 j of a token in registers (E <= 256,
+// groups of a multiple of 32 experts, T K <= 32).  Per token: group score =
+// sum of the two largest biased scores (warp max reductions); the TG best
+// groups kept (ties to the lower group); then each lane sorts its kept
+// candidates (larger biased score, then lower index) and K rounds of a warp
+// arg-max over the lanes' best remaining candidate give the slots in order.
+// Gate weights use the unbiased scores, their sum taken in slot order.  The
+// union lists the pairs by (expert, token).  Runs on the helper warp, in
+// parallel with the consumers, which never wait for it; the producer waits on
+// route_bar.
+__device__ __forceinline__ void route_warp(const FusedParams& p, const Smem& s) {
+    constexpr int NJ = kMaxExpertsPerLane;
+    const int lane = threadIdx.x & 31;
+    const int T = p.T, K = p.K, E = p.E, G = p.G, TG = p.TG, NE = E >> 5, m = NE / G;
+    const uint32_t tag = *s.tag;
+    float bias_r[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) bias_r[j] = j < NE ? __ldg(p.bias + lane + 32 * j) : 0.0f;
+    bool ok = true;
+    int pe = 0;  // lane t K + k: expert of token t, slot k
+    float pw = 0.0f;
+    for (int t = 0; t < T; ++t) {
+        // this token's scores, as soon as every slot carries this launch's tag
+        float sc[NJ];
+        uint32_t pend = (1u << NE) - 1u;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) sc[j] = 0.0f;
+        for (long it = 0; ok; ++it) {
+            // all loads first (their predicates must not depend on earlier
+            // loads' results, or they would be issued one after another)
+            unsigned long long v[NJ];
+            const uint32_t want = pend;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+                v[j] = ((want >> j) & 1u) ? ld_relaxed_gpu_u64(p.scores + t * E + lane + 32 * j) : 0ull;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) {
+                if (((want >> j) & 1u) && static_cast<uint32_t>(v[j] >> 32) == tag) {
+                    sc[j] = __uint_as_float(static_cast<uint32_t>(v[j]));
+                    pend &= ~(1u << j);
+                }
             }
+            if (__all_sync(0xffffffffu, pend == 0)) break;
+            if (it >= kProducerWait) ok = false;
             __nanosleep(32);
         }
-        if (!okc) record_status(p.status, MOE_EDEVICE_TIMEOUT);
-    }
-    consumers_sync();
-    for (int i = tid; i < T * E; i += kConsumers) {
-        const int e = i % E;
-        const double l = static_cast<double>(__ldcg(p.logits + i));
-        const float sc = __double2float_rn(1.0 / (1.0 + exp(-l)));
-        sv[i] = sc;
-        bv[i] = __fadd_rn(sc, s.bias[e]);
-    }
-    for (int i = tid; i < T * 32; i += kConsumers) ch[i] = -1;
-    if (tid < 32) s.bmap[tid] = 0;
-    consumers_sync();
-    // group scores: one warp per (token, group); lane-local top-2, then a warp merge
-    for (int pg = warp; pg < T * G; pg += kConsumerWarps) {
-        const int t = pg / G, g = pg % G;
-        const float* bg = bv + t * E + g * gsz;
-        float m1 = -INFINITY, m2 = -INFINITY;
-        for (int e = lane; e < gsz; e += 32) {
-            const float v = bg[e];
-            if (v > m1) {
-                m2 = m1;
-                m1 = v;
-            } else if (v > m2) {
-                m2 = v;
-            }
-        }
+        uint32_t key[NJ];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float o1 = __shfl_xor_sync(0xffffffffu, m1, o), o2 = __shfl_xor_sync(0xffffffffu, m2, o);
-            const float n1 = fmaxf(m1, o1);
-            m2 = fmaxf(fminf(m1, o1), fmaxf(m2, o2));
-            m1 = n1;
-        }
-        if (lane == 0) gs[pg] = __fadd_rn(m1, m2);
-    }
-    consumers_sync();
-    // kept groups: rank each group's score among its token's groups
-    for (int i = tid; i < T * G; i += kConsumers) {
-        const int t = i / G, g = i % G;
-        const float v = gs[i];
-        int r = 0;
-        for (int g2 = 0; g2 < G; ++g2) {
-            const float w = gs[t * G + g2];
-            r += (w > v) || (w == v && g2 < g);
-        }
-        if (r < TG) kg[t * TG + r] = g;
-    }
-    consumers_sync();
-    // experts: rank each expert of a kept group among all experts of kept groups
-    for (int i = tid; i < T * E; i += kConsumers) {
-        const int t = i / E, e = i % E, ge = e / gsz;
-        bool kept = false;
-        for (int j = 0; j < TG; ++j) kept |= kg[t * TG + j] == ge;
-        if (!kept) continue;
-        const float v = bv[i];
-        int r = 0;
-        for (int j = 0; j < TG; ++j) {
-            const int base = kg[t * TG + j] * gsz;
-            const float* bg = bv + t * E + base;
-            if (vec) {
-                const float4* bg4 = reinterpret_cast<const float4*>(bg);
-#pragma unroll 4
-                for (int q = 0; q < gsz / 4; ++q) {
-                    const float4 w = bg4[q];
-                    const int x = base + 4 * q;
-                    r += (w.x > v) | ((w.x == v) & (x < e));
-                    r += (w.y > v) | ((w.y == v) & (x + 1 < e));
-                    r += (w.z > v) | ((w.z == v) & (x + 2 < e));
-                    r += (w.w > v) | ((w.w == v) & (x + 3 < e));
-                }
+        for (int j = 0; j < NJ; ++j) key[j] = j < NE ? order_key(__fadd_rn(sc[j], bias_r[j])) : 0u;
+        // group g = rows j in [g m, g m + m): the two largest keys of the
+        // group (equal maxima in two lanes count twice), summed as values
+        float gsum[NJ];
+#pragma unroll
+        for (int g = 0; g < NJ; ++g) {
+            uint32_t k1 = 0, k2 = 0;
+            if (m == 1) {  // one row per group (32 experts)
+                k1 = g < G ? key[g] : 0u;
             } else {
-                for (int q = 0; q < gsz; ++q) r += (bg[q] > v) | ((bg[q] == v) & (base + q < e));
-            }
-        }
-        if (r < K) ch[t * 32 + r] = e;
-    }
-    consumers_sync();
-    // per token (warp t, lane k = slot): guard, gate weight, entry, bitmap
-    if (warp < T) {
-        const int t = warp;
-        int e = lane < K ? ch[t * 32 + lane] : 0;
-        if (lane < K && (e < 0 || e >= E)) {  // only reachable with NaN scores
-            record_status(p.status, MOE_EDEVICE_INDEX);
-            e = 0;
-        }
-        const float sk = lane < K ? sv[t * E + e] : 0.0f;
-        float den = 0.0f;  // sum in slot order, as the definition orders it
-        for (int j = 0; j < K; ++j) den = __fadd_rn(den, __shfl_sync(0xffffffffu, sk, j));
-        if (lane < K) {
-            ch[t * 32 + lane] = e;
-            s.rt_w[t * K + lane] = __fmul_rn(__fdiv_rn(sk, den), p.rsf);
-            s.ent[t * K + lane] = e;
-            atomicOr(&s.bmap[e >> 5], 1u << (e & 31));
-        }
-    }
-    consumers_sync();
-    if (warp == 0) {  // exclusive prefix of the bitmap's popcounts
-        const int c = __popc(s.bmap[lane]);
-        int incl = c;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n2 = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += n2;
+                for (int j = 0; j < NJ; ++j) {
+                    if (g < G && j >= g * m && j < g * m + m) {
+                        k2 = max(k2, min(k1, key[j]));
+                        k1 = max(k1, key[j]);
+                    }
+                }
+            }
+            const uint32_t m1 = __reduce_max_sync(0xffffffffu, k1);
+            const uint32_t at = __ballot_sync(0xffffffffu, k1 == m1);
+            const uint32_t r2 = __reduce_max_sync(0xffffffffu, (k1 == m1 && (at & ((1u << lane) - 1u)) == 0) ? k2 : k1);
+            gsum[g] = __fadd_rn(key_value(m1), key_value(r2));
         }
-        bpre[lane] = incl - c;
-        if (lane == 31) bpre[32] = incl;
-    }
-    consumers_sync();
-    // union of the T*K entries: (expert ascending, token ascending) positions
-    const int n = T * K;
-    for (int i = tid; i < n; i += kConsumers) {
-        const int t = i / K, e = s.ent[i];
-        int before = 0, same_before = 0, first = 1;
-        for (int jx = 0, tj = 0, kj = 0; jx < n; ++jx) {  // tj = jx / K without a division
-            const int ej = s.ent[jx];
-            before += ej < e;
-            same_before += (ej == e) & (tj < t);
-            first &= !((ej == e) & (jx < i));
-            if (++kj == K) {
-                kj = 0;
-                ++tj;
+        // kept groups: each lane ranks group `lane` against the others
+        float mine = 0.0f;
+#pragma unroll
+        for (int g = 0; g < NJ; ++g)
+            if (g == lane) mine = gsum[g];
+        int r = 0;
+#pragma unroll
+        for (int g = 0; g < NJ; ++g) r += g < G && ((gsum[g] > mine) || (gsum[g] == mine && g < lane));
+        const uint32_t kept = __ballot_sync(0xffffffffu, lane < G && r < TG);
+        uint32_t kept_rows = 0;  // rows j of the kept groups
+#pragma unroll
+        for (int g = 0; g < NJ; ++g)
+            if (g < G && ((kept >> g) & 1u)) kept_rows |= ((1u << m) - 1u) << (g * m);
+        // this lane's candidates of the kept groups, sorted (best first) by an
+        // optimal 19-comparator network for 8 inputs
+        uint32_t ck[NJ];
+        int ce[NJ];
+        float cs[NJ];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+            ck[j] = ((kept_rows >> j) & 1u) ? key[j] : 0u;
+            ce[j] = lane + 32 * j;
+            cs[j] = sc[j];
+        }
+        static_assert(NJ == 8, "sorting network is for 8 candidates");
+        constexpr int kNet[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6}, {5, 7}, {1, 2}, {5, 6},
+                                     {0, 4}, {3, 7}, {1, 5}, {2, 6}, {1, 4}, {3, 6}, {2, 4}, {3, 5}, {3, 4}};
+#pragma unroll
+        for (int c = 0; c < 19; ++c) {
+            const int a = kNet[c][0], b = kNet[c][1];
+            cand_order(ck[a], ce[a], cs[a], ck[b], ce[b], cs[b]);
+        }
+        // K rounds: the warp's best head wins; its lane pops it
+        int my_e = -1;
+        float my_s = 0.0f, den = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            const uint32_t mx = __reduce_max_sync(0xffffffffu, ck[0]);
+            const uint32_t win = __reduce_min_sync(0xffffffffu, (ck[0] == mx && mx != 0u) ? static_cast<uint32_t>(ce[0]) : 0xffffffffu);
+            const bool mine_w = static_cast<uint32_t>(ce[0]) == win;
+            const float sw = __shfl_sync(0xffffffffu, cs[0], win & 31u);
+            den = __fadd_rn(den, sw);  // slot order
+            if (lane == k) {
+                my_e = static_cast<int>(win);
+                my_s = sw;
+            }
+            if (mine_w) {
+#pragma unroll
+                for (int j = 0; j < NJ - 1; ++j) {
+                    ck[j] = ck[j + 1];
+                    ce[j] = ce[j + 1];
+                    cs[j] = cs[j + 1];
+                }
+                ck[NJ - 1] = 0u;
             }
         }
-        const int rank = bpre[e >> 5] + __popc(s.bmap[e >> 5] & ((1u << (e & 31)) - 1u));
-        const int pos = before + same_before;
-        s.rt_ptok[pos] = t;
-        s.rt_pair_of[i] = pos;
+        if (lane < K && (my_e < 0 || my_e >= E)) {  // only reachable with NaN scores
+            record_status(p.status, MOE_EDEVICE_INDEX);
+            my_e = 0;
+        }
+        const float my_w = __fmul_rn(__fdiv_rn(my_s, den), p.rsf);
+        // move token t's K results to lanes t K .. t K + K - 1
+        const int src = lane - t * K;
+        const int e_t = __shfl_sync(0xffffffffu, my_e, src & 31);
+        const float w_t = __shfl_sync(0xffffffffu, my_w, src & 31);
+        if (src >= 0 && src < K) {
+            pe = e_t;
+            pw = w_t;
+        }
+    }
+    if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
+    // batch union: pair position = number of pairs with a smaller (expert, token)
+    const int n = T * K;  // <= 32
+    const bool act = lane < n;
+    const int key = act ? (pe << 5) | lane : 0x7fffffff;
+    const uint32_t same = T > 1 ? __match_any_sync(0xffffffffu, act ? pe : -1 - lane) : (1u << lane);
+    const bool first = act && (__ffs(same) - 1 == lane);
+    const uint32_t firsts = __ballot_sync(0xffffffffu, first);
+    int pos = 0, urank = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int kj = __shfl_sync(0xffffffffu, key, j);
+        if (j < n) {
+            pos += kj < key;
+            urank += ((firsts >> j) & 1u) && (kj >> 5) < pe;
+        }
+    }
+    if (act) {
+        s.rt_ptok[pos] = lane / K;
+        s.rt_pair_of[lane] = pos;
+        s.rt_w[lane] = pw;
         if (first) {
-            s.rt_uniq[rank] = e;
-            s.rt_off[rank] = before;
+            s.rt_uniq[urank] = pe;
+            s.rt_off[urank] = pos;
+        }
+        if (blockIdx.x == 0) {  // the routing the caller can see, written once
+            p.idx[lane] = pe;
+            p.w[lane] = pw;
         }
     }
-    if (tid == 0) {
-        const int U = bpre[32];
-        *s.rt_U = U;
-        s.rt_off[U] = n;
+    if (lane == 0) {
+        *s.rt_U = __popc(firsts);
+        s.rt_off[__popc(firsts)] = n;
     }
-    consumers_sync();
-    if (tid == 0) mbar_arrive(s.route_bar);
-    // the routing outputs the caller can see, written once (off the critical path)
-    if (blockIdx.x == 0) {
-        for (int i = tid; i < n; i += kConsumers) {
-            p.idx[i] = ch[(i / K) * 32 + (i % K)];
-            p.w[i] = s.rt_w[i];
-        }
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(s.route_bar);
 }
 
 // Activations of one token for the blocks a lane owns (b = lane + 32 j), in registers.
@@ -945,7 +989,7 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
     }
 }
 
-// Hands a finished tile (or the end) to the epilogue warp through task slot tb.
+// Hands a finished tile (or the end) to epilogue warp tb through task slot tb.
 __device__ __forceinline__ void push_task(const Smem& s, int tb, const Desc* d, int type) {
     const int tid = threadIdx.x, lane = tid & 31;
     if (tid == 0) {
@@ -988,7 +1032,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
             phase ^= 1u;
         }
     };
-    // Waits until the epilogue warp has finished with task slot tb.
+    // Waits until epilogue warp tb has finished with task slot tb.
     auto task_slot_free = [&]() -> bool {
         if (!mbar_wait(&s.tfree[tb], tph[tb] ^ 1u, kConsumerWait)) {
             record_status(p.status, MOE_EDEVICE_TIMEOUT);
@@ -1001,7 +1045,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
         tb ^= 1;
     };
     int type = next_type();
-    // phase A: router rows, then (at the route marker) Q8_0 of x and the routing
+    // phase A: router rows (the helper warp routes meanwhile), then Q8_0 of x
     while (type == D_ROUTER) {
         const int e0 = s.desc[stage].e, nrows = s.desc[stage].nrows;
         consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes);
@@ -1010,106 +1054,152 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     }
     quantize_x<QT>(p, s);
     consumers_sync();
-    if (type == D_ROUTE) {
-        route_cta(p, s);
-        release();
-        type = next_type();
-    }
-    // phase B: up/gate tiles
+    // phases B and C: runs of up/gate tiles and of down tiles, interleaved
     bool ok = true;
-    {
-        ActRegs<kRegChunksUg> ar;
-        if constexpr (NT == 1) {
-            const int nbH = p.H / 32;
-#pragma unroll
-            for (int j = 0; j < kRegChunksUg; ++j) {
-                const int b = lane + 32 * j;
-                ar.a0[j] = b < nbH ? s.q0[b] : make_uint4(0, 0, 0, 0);
-                ar.a1[j] = b < nbH ? s.q1[b] : make_uint4(0, 0, 0, 0);
-            }
-        }
-        while (type == D_UG) {
-            const Desc& d = s.desc[stage];
-            const uint8_t* sbuf = s.ring + stage * slot_bytes;
-            if (d.first && !task_slot_free()) {
-                ok = false;
-                break;
-            }
-            float* dst = (d.mat == 0 ? s.gbuf : s.ubuf) + tb * kMaxT * kUgTileRows;
+    while (ok && (type == D_UG || type == D_DOWN)) {
+        if (type == D_UG) {
+            // NT = 1: the token's Q8_0 x lives in registers for the run
+            ActRegs<kRegChunksUg> ar;
             if constexpr (NT == 1) {
-                consume_ug_reg<QT>(p, s, dst, d.row0, sbuf, ar);
-            } else {
-                consume_ug_smem<QT, NT>(p, s, d, dst, sbuf);
+                const int nbH = p.H / 32;
+#pragma unroll
+                for (int j = 0; j < kRegChunksUg; ++j) {
+                    const int b = lane + 32 * j;
+                    ar.a0[j] = b < nbH ? s.q0[b] : make_uint4(0, 0, 0, 0);
+                    ar.a1[j] = b < nbH ? s.q1[b] : make_uint4(0, 0, 0, 0);
+                }
             }
-            if (d.last) {
-                push_task(s, tb, &d, D_UG);
-                next_task();
-            }
-            release();
-            type = next_type();
-        }
-    }
-    // phase C: down tiles
-    if (ok) {
-        ActRegs<kRegChunksDown> ar;
-        const float* ad = nullptr;
-        const int32_t* as = nullptr;
-        while (type == D_DOWN) {
-            const Desc& d = s.desc[stage];
-            const uint8_t* sbuf = s.ring + stage * slot_bytes;
-            if (d.first) {
-                if (!mbar_wait(&s.afull[aslot], aphase, kConsumerWait)) {
-                    record_status(p.status, MOE_EDEVICE_TIMEOUT);
+            while (type == D_UG) {
+                const Desc& d = s.desc[stage];
+                const uint8_t* sbuf = s.ring + stage * slot_bytes;
+                if (d.first && !task_slot_free()) {
+                    ok = false;
                     break;
                 }
+                float* dst = (d.mat == 0 ? s.gbuf : s.ubuf) + tb * kMaxT * kUgTileRows;
                 if constexpr (NT == 1) {
-                    const uint8_t* rec = s.act + static_cast<size_t>(aslot) * p.act_bytes;
-                    const int nbI = p.I / 32;
-#pragma unroll
-                    for (int j = 0; j < kRegChunksDown; ++j) {
-                        const int b = lane + 32 * j;
-                        ar.a0[j] = b < nbI ? reinterpret_cast<const uint4*>(rec)[b] : make_uint4(0, 0, 0, 0);
-                        ar.a1[j] = b < nbI ? reinterpret_cast<const uint4*>(rec + p.I / 2)[b]
-                                           : make_uint4(0, 0, 0, 0);
+                    consume_ug_reg<QT>(p, s, dst, d.row0, sbuf, ar);
+                } else {
+                    consume_ug_smem<QT, NT>(p, s, d, dst, sbuf);
+                }
+                if (d.last) {
+                    push_task(s, tb, &d, D_UG);
+                    next_task();
+                }
+                release();
+                type = next_type();
+            }
+        } else {
+            ActRegs<kRegChunksDown> ar;
+            const float* ad = nullptr;
+            const int32_t* as = nullptr;
+            while (type == D_DOWN) {
+                const Desc& d = s.desc[stage];
+                const uint8_t* sbuf = s.ring + stage * slot_bytes;
+                if (d.first) {
+                    if (!mbar_wait(&s.afull[aslot], aphase, kConsumerWait)) {
+                        record_status(p.status, MOE_EDEVICE_TIMEOUT);
+                        ok = false;
+                        break;
                     }
-                    ad = reinterpret_cast<const float*>(rec + p.I);
-                    as = reinterpret_cast<const int32_t*>(rec + p.I + nbI * 4);
+                    if constexpr (NT == 1) {
+                        const uint8_t* rec = s.act + static_cast<size_t>(aslot) * p.act_bytes;
+                        const int nbI = p.I / 32;
+#pragma unroll
+                        for (int j = 0; j < kRegChunksDown; ++j) {
+                            const int b = lane + 32 * j;
+                            ar.a0[j] = b < nbI ? reinterpret_cast<const uint4*>(rec)[b] : make_uint4(0, 0, 0, 0);
+                            ar.a1[j] = b < nbI ? reinterpret_cast<const uint4*>(rec + p.I / 2)[b]
+                                               : make_uint4(0, 0, 0, 0);
+                        }
+                        ad = reinterpret_cast<const float*>(rec + p.I);
+                        as = reinterpret_cast<const int32_t*>(rec + p.I + nbI * 4);
+                    }
                 }
-            }
-            if constexpr (NT == 1) {
-                consume_down_reg<QT>(p, d.row0, d.nrows, d.pair[0], sbuf, ar, ad, as);
-            } else {
-                consume_down_smem<QT, NT>(p, s, d, sbuf);
-            }
-            if (d.last) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.aempty[aslot]);
-                if (++aslot == kActSlots) {
-                    aslot = 0;
-                    aphase ^= 1u;
+                if constexpr (NT == 1) {
+                    consume_down_reg<QT>(p, d.row0, d.nrows, d.pair[0], sbuf, ar, ad, as);
+                } else {
+                    consume_down_smem<QT, NT>(p, s, d, sbuf);
                 }
-                if (!task_slot_free()) break;
-                push_task(s, tb, &d, D_DOWN);
-                next_task();
+                if (d.last) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.aempty[aslot]);
+                    if (++aslot == kActSlots) {
+                        aslot = 0;
+                        aphase ^= 1u;
+                    }
+                    if (!task_slot_free()) {
+                        ok = false;
+                        break;
+                    }
+                    push_task(s, tb, &d, D_DOWN);
+                    next_task();
+                }
+                release();
+                type = next_type();
             }
-            release();
-            type = next_type();
         }
     }
-    // hand the end to the epilogue warp
-    if (task_slot_free()) push_task(s, tb, nullptr, D_EXIT);
+    // hand the end to both epilogue warps
+    for (int i = 0; i < kTaskSlots; ++i) {
+        if (!task_slot_free()) break;
+        push_task(s, tb, nullptr, D_EXIT);
+        next_task();
+    }
+}
+
+// ------------------------------------------------------------------ helper warp
+// Routes the batch (all lanes), then lane 0 serves the producer's down-tile
+// requests in order: waits until the slot's previous records are consumed and
+// the expert's h tiles are all complete, then bulk-copies the records.
+template <int QT>
+__device__ __forceinline__ void helper_warp(const FusedParams& p, const Smem& s) {
+    route_warp(p, s);
+    if ((threadIdx.x & 31) != 0) return;
+    long n_act = 0;
+    int slot = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    while (true) {
+        if (!mbar_wait(&s.areq_full[slot], ph, kProducerWait)) {
+            ok = false;
+            break;
+        }
+        const ActReq rq = s.areq[slot];
+        if (rq.exit) break;
+        if (!mbar_wait(&s.aempty[slot], ph ^ 1u, kProducerWait) ||
+            !wait_counter_geq(p.ug_done + rq.cslot, rq.need, kProducerWait)) {
+            ok = false;
+            break;
+        }
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&s.afull[slot], rq.bytes);
+        bulk_g2s(s.act + static_cast<size_t>(slot) * p.act_bytes, rq.src, rq.bytes, &s.afull[slot]);
+        ++n_act;
+        mbar_arrive(&s.areq_free[slot]);
+        if (++slot == kActSlots) {
+            slot = 0;
+            ph ^= 1u;
+        }
+    }
+    if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
+    // drain: every record copy issued into this CTA's shared memory has landed
+    for (int a = 0; a < kActSlots; ++a) {
+        const long uses = n_act / kActSlots + (a < n_act % kActSlots ? 1 : 0);
+        if (uses > 0) mbar_wait(&s.afull[a], static_cast<uint32_t>((uses - 1) & 1), kProducerWait);
+    }
 }
 
 // ------------------------------------------------------------------ epilogue warp
 template <int QT>
-__device__ void epilogue_warp(const FusedParams& p, const Smem& s) {
+__device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
+    // epilogue warp tb serves task slot tb
     const int lane = threadIdx.x & 31;
     const int nbI = p.I / 32;
     const int P = p.T * p.K;
-    int tb = 0;
-    uint32_t eph[kTaskSlots] = {0, 0};
+    uint32_t eph = 0;
     while (true) {
-        if (!mbar_wait(&s.tfull[tb], eph[tb], kEpilogueWait)) {
+        if (!mbar_wait(&s.tfull[tb], eph, kEpilogueWait)) {
             record_status(p.status, MOE_EDEVICE_TIMEOUT);
             break;
         }
@@ -1162,8 +1252,7 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s) {
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.tfree[tb]);
-        eph[tb] ^= 1u;
-        tb ^= 1;
+        eph ^= 1u;
     }
 }
 
@@ -1195,13 +1284,20 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfree[i], 1);
         }
         mbar_init(s.route_bar, 1);
+        for (int i = 0; i < kActSlots; ++i) {
+            mbar_init(&s.areq_full[i], 1);
+            mbar_init(&s.areq_free[i], 1);
+        }
         fence_mbar_init();
+        *s.tag = static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch))) + 1u;
     }
     __syncthreads();
     if (warp == kProducerWarp) {
         if (lane == 0) producer<QT>(p, s);
-    } else if (warp == kEpilogueWarp) {
-        epilogue_warp<QT>(p, s);
+    } else if (warp == kHelperWarp) {
+        helper_warp<QT>(p, s);
+    } else if (warp >= kEpilogueWarp0) {
+        epilogue_warp<QT>(p, s, warp - kEpilogueWarp0);
     } else {
         consumer<QT, NT>(p, s);
     }
@@ -1213,9 +1309,8 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             for (int i = 0; i <= p.E; ++i) p.ug_done[i] = 0;
             for (int i = 0; i < p.n_dt; ++i) p.rb_done[i] = 0;
             p.sync->ticket = 0;
-            p.sync->router_done = 0;
-            p.sync->route_ready = 0;
             p.sync->exit_count = 0;
+            *p.epoch = *s.tag;
             __threadfence();
         }
     }
@@ -1230,9 +1325,11 @@ const void* fused_kernel(int nt) {
 }  // namespace
 
 bool fused_geometry(FusedParams& p, int qtype) {
-    // the routing scratch (scores, biased scores, group scores and flags of
-    // every token) reuses the bf16 copy of x: needs 6 E <= H
-    if (p.T < 1 || p.T > kMaxT || p.K * p.T > 128 || 6 * p.E > p.H) return false;
+    // one warp routes the batch: experts lane + 32 j in registers (E <= 256),
+    // groups of a multiple of 32 experts, the batch's T K pairs in one warp
+    if (p.T < 1 || p.T > kMaxT || p.K < 1 || p.K * p.T > 32 || p.T * p.E > kFusedMaxSlots) return false;
+    if (p.E % 32 || p.E > 32 * kMaxExpertsPerLane || p.G < 1 || p.E % p.G || (p.E / p.G) % 32) return false;
+    if (p.TG < 1 || p.TG > p.G || p.TG * (p.E / p.G) < p.K) return false;
     const size_t rb_ug = static_cast<size_t>(p.H) * qtype / 8, rb_d = static_cast<size_t>(p.I) * qtype / 8;
     size_t stage = std::max(static_cast<size_t>(4) * p.H, kStageRows * rb_ug);
     stage = (stage + 127) / 128 * 128;

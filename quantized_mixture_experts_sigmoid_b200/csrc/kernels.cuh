@@ -53,19 +53,27 @@ cudaError_t launch_combine(const float* y, const float* w, const float* shared_y
 // ------------------------------------------------------------ fused small-batch layer
 constexpr int kFusedMaxTokens = 4;
 
-// Control block at the start of every workspace (kWsHeader bytes, zero when idle).
+// Control block at the start of every workspace (kWsHeader bytes).  The
+// counters before kWsScoresOff are zero when idle.  The score slots hold the
+// router scores of the last launch, each tagged with its launch number; the
+// word at kWsEpochOff counts the fused kernel's launches on this workspace and
+// is never cleared, so a slot written by an earlier launch (or zeroed by a
+// status clear) never carries the current launch's tag.  Nothing but the
+// fused kernel writes the slots.
 struct FusedSync {
     int ticket;
-    int router_done;
-    int route_ready;
     int exit_count;
-    int pad[12];
+    int pad[14];
 };
 constexpr size_t kWsStatusOff = 0;
 constexpr size_t kWsSyncOff = 64;
 constexpr size_t kWsUgDoneOff = 128;                    // int[E + 1], E <= 1024
 constexpr size_t kWsRbDoneOff = kWsUgDoneOff + 4 * 1032; // int[n_dt], n_dt <= 16384 / 32 + 1
-static_assert(kWsRbDoneOff + 4 * 520 <= kWsHeader, "workspace header too small");
+constexpr size_t kWsScoresOff = 6400;                   // u64[T * E], T * E <= kFusedMaxSlots
+constexpr int kFusedMaxSlots = 1024;
+constexpr size_t kWsEpochOff = kWsHeader - 64;
+static_assert(kWsRbDoneOff + 4 * 520 <= kWsScoresOff, "workspace header too small");
+static_assert(kWsScoresOff + 8 * kFusedMaxSlots <= kWsEpochOff, "workspace header too small");
 
 struct FusedParams {
     const uint16_t* x;
@@ -84,7 +92,8 @@ struct FusedParams {
     FusedSync* sync;
     int32_t* ug_done;
     int32_t* rb_done;
-    float* logits;
+    uint32_t* epoch;                 // launch counter (workspace header, never cleared)
+    unsigned long long* scores;      // [T][E] router scores, low word fp32 bits, high word launch tag
     int32_t* n_unique;
     int32_t* uniq;
     int32_t* offsets;

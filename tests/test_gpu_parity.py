@@ -29,13 +29,14 @@ SHAPES = {
                                      topk_group=2, top_k=5, qtype=8),
     "crowded_int2": synth.LayerShape("crowded_int2", T=100, H=544, I=288, E=16, n_group=4,
                                      topk_group=2, top_k=5, qtype=2),
-    # small batches take the fused persistent kernel: ragged shapes, T = 2 and 3
-    "fused_ragged": synth.LayerShape("fused_ragged", T=3, H=544, I=288, E=48, n_group=6, topk_group=3,
+    # small batches take the fused persistent kernel (groups of a multiple of
+    # 32 experts): ragged hidden sizes, T = 2, 3 and 4, 1 to 4 groups
+    "fused_ragged": synth.LayerShape("fused_ragged", T=3, H=544, I=288, E=64, n_group=2, topk_group=1,
                                      top_k=5),
-    "fused_ragged_int2": synth.LayerShape("fused_ragged_int2", T=2, H=576, I=160, E=64, n_group=8,
+    "fused_ragged_int2": synth.LayerShape("fused_ragged_int2", T=2, H=576, I=160, E=128, n_group=4,
                                           topk_group=2, top_k=6, qtype=2),
-    "fused_ragged_int8": synth.LayerShape("fused_ragged_int8", T=4, H=544, I=288, E=48, n_group=6,
-                                          topk_group=3, top_k=5, qtype=8),
+    "fused_ragged_int8": synth.LayerShape("fused_ragged_int8", T=4, H=544, I=288, E=96, n_group=3,
+                                          topk_group=2, top_k=5, qtype=8),
     "decode": synth.CONFIGS["decode"],
     "verify": synth.CONFIGS["verify"],
     "verify_int8": synth.CONFIGS["verify_int8"],
@@ -277,6 +278,29 @@ def test_union_path_equals_per_token_path_on_gpu():
         assert np.array_equal(of_one.view(np.uint32), of_batch[t:t + 1].view(np.uint32))
 
 
+FUSED = ["fused_ragged", "fused_ragged_int2", "fused_ragged_int8", "decode", "verify", "decode_int2"]
+
+
+@pytest.mark.parametrize("name", FUSED + ["tiny", "ragged"])
+def test_layer_forward_path(name):
+    # small batches with groups of a multiple of 32 experts run as one fused
+    # launch; other shapes take the multi-kernel path
+    sh, dev = layer(name)
+    x, W, b = layer_inputs(sh)
+    xd = to_dev_bf16(x)
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
+    out = torch.empty(sh.T, sh.H, dtype=torch.float32, device="cuda")
+    n0 = moe.lib().moe_launch_count()
+    moe.moe_layer_forward(xd, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+    torch.cuda.synchronize()
+    n = moe.lib().moe_launch_count() - n0
+    assert moe.moe_workspace_status(ws) == 0
+    if name in FUSED:
+        assert n == 1
+    else:
+        assert n > 1
+
+
 def test_layer_forward_repeated_calls_reuse_workspace():
     # the fused kernel's counters live in the workspace and reset themselves:
     # many calls in a row on one workspace give the same, correct result
@@ -289,6 +313,13 @@ def test_layer_forward_repeated_calls_reuse_workspace():
         out = torch.empty(sh.T, sh.H, dtype=torch.float32, device="cuda")
         moe.moe_layer_forward(xd, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
         outs.append(out)
+    torch.cuda.synchronize()
+    assert moe.moe_workspace_status(ws) == 0  # also clears the counters
+    # after a status clear the launch counter carries on: stale score slots of
+    # earlier calls are never taken for this call's
+    out = torch.empty(sh.T, sh.H, dtype=torch.float32, device="cuda")
+    moe.moe_layer_forward(xd, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+    outs.append(out)
     torch.cuda.synchronize()
     assert moe.moe_workspace_status(ws) == 0
     first = outs[0].cpu().numpy()
