@@ -52,6 +52,27 @@ def peaks():
         return 6650.0, "fallback"
 
 
+KERNEL_SOURCES = ("decode_fused.cu", "common.cuh", "kernels.cuh", "quant.cuh", "sm100_async.cuh")
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None when
+    the kernel sources have changed since that capture."""
+    import hashlib
+    import re
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "k_decode_fused_decode.md")).read()
+        traffic = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt).group(1))
+        sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt).group(1)
+    except (OSError, AttributeError):
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "quantized_mixture_experts_sigmoid_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return traffic if h.hexdigest() == sha else None
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -286,7 +307,7 @@ def run_cuda(args):
         "frac_of_8TBps": layer_bytes / (ms_step / 1e3) / 1e9 / NOMINAL_HBM_GBS,
         "roofline": {"bound": "hbm", "kernel": "k_decode_fused (whole layer, one launch)",
                      "achieved": dom_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": None,
+                     "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": profiled_traffic(),
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
         "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},

@@ -59,17 +59,20 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kGroups = 2;  // consumer groups: ring stage n belongs to group n % kGroups
+constexpr int kGroupWarps = kConsumerWarps / kGroups;
+constexpr int kGroupThreads = kGroupWarps * 32;
 constexpr int kEpilogueWarps = 2;    // one per task slot
 constexpr int kEpilogueWarp0 = kConsumerWarps;
 constexpr int kProducerWarp = kEpilogueWarp0 + kEpilogueWarps;
 constexpr int kHelperWarp = kProducerWarp + 1;  // routing, then the activation copies
 constexpr int kThreadsF = (kHelperWarp + 1) * 32;
 constexpr int kMaxT = kFusedMaxTokens;
-constexpr int kStageRows = 16;       // up/gate rows per stage (one per consumer warp)
+constexpr int kStageRows = 16;       // up/gate rows per stage (two per warp of a group)
 constexpr int kUgTileRows = 32;      // one Q8_0 block of h
-constexpr int kDownStagesPerTile = 2;
+constexpr int kDownStagesPerTile = 2;  // one per consumer group
 constexpr int kMaxRouterRows = 4;    // router rows per stage
-constexpr int kMaxDownRowsPerWarp = 4;
+constexpr int kMaxDownRowsPerWarp = 8;
 constexpr int kActSlots = 2;
 constexpr int kTaskSlots = kEpilogueWarps;
 constexpr int kScaleBytes = 256;     // room after each stage for its rows' fp32 scales
@@ -82,7 +85,10 @@ constexpr int kRegChunksDown = 2;    // NT = 1: blocks of h per lane held in reg
 constexpr long kProducerWait = 1L << 22;
 constexpr long kConsumerWait = 1L << 24;
 constexpr long kEpilogueWait = 1L << 25;
-constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps
+constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps (group g: 2 + g)
+static_assert(kStageRows == 2 * kGroupWarps, "an up/gate stage gives each warp of a group two rows");
+static_assert(kDownStagesPerTile == kGroups && (2 * (kUgTileRows / kStageRows)) % kGroups == 0,
+              "the stages of every tile reach every consumer group");
 constexpr int kDownLag = 8;          // routed experts between an expert's up/gate and down tiles
 constexpr int kMaxExpertsPerLane = 8; // warp routing: E <= 32 * 8
 
@@ -99,6 +105,8 @@ struct Desc {
     int first;
     int last;
     int blk;        // up/gate: h block index; down: row block index
+    int sit;        // stage index within its tile
+    int nst;        // stages in the tile (4 up/gate, 2 down: every group sees every tile)
     int aslot;
     int n_experts;  // shared + distinct routed experts (down tiles)
     int n_tok;
@@ -244,6 +252,7 @@ __device__ __forceinline__ WBlock<QT> load_wblock_smem(const uint8_t* row, int b
 }
 
 __device__ __forceinline__ void consumers_sync() { named_bar_sync(kBarConsumers, kConsumers); }
+__device__ __forceinline__ void group_sync(int g) { named_bar_sync(kBarConsumers + 1 + g, kGroupThreads); }
 
 // Element of a 32-block that byte i of permuted activation word w holds,
 // matching the field order in which block_dot<QT> presents weight codes.
@@ -335,9 +344,13 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         if (!acquire_stage()) return false;
         s.desc[stage] = d;
         uint8_t* dst = s.ring + stage * slot_bytes;
-        mbar_arrive_expect_tx(&s.full[stage], w_bytes + s_bytes);
-        bulk_g2s_hint(dst, w_src, w_bytes, &s.full[stage], pol);
-        if (s_bytes) bulk_g2s(dst + p.stage_bytes, s_src, s_bytes, &s.full[stage]);
+        if (w_bytes == 0) {  // an empty stage (the short half of a ragged down tile)
+            mbar_arrive(&s.full[stage]);
+        } else {
+            mbar_arrive_expect_tx(&s.full[stage], w_bytes + s_bytes);
+            bulk_g2s_hint(dst, w_src, w_bytes, &s.full[stage], pol);
+            if (s_bytes) bulk_g2s(dst + p.stage_bytes, s_src, s_bytes, &s.full[stage]);
+        }
         advance();
         return true;
     };
@@ -400,6 +413,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         if (kind == 0) {  // up/gate tile: rows 32j..32j+31 of gate, then of up
             d.type = D_UG;
             d.nrows = kStageRows;
+            d.nst = 2 * (kUgTileRows / kStageRows);
             for (int m = 0; m < 2 && ok; ++m) {
                 const uint8_t* wm = m == 0 ? ex.w_gate : ex.w_up;
                 const float* sm = m == 0 ? ex.s_gate : ex.s_up;
@@ -408,6 +422,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                     d.row0 = j * kUgTileRows + q * kStageRows;
                     d.first = (m == 0 && q == 0);
                     d.last = (m == 1 && q == kUgTileRows / kStageRows - 1);
+                    d.sit = m * (kUgTileRows / kStageRows) + q;
                     const size_t r = static_cast<size_t>(d.e) * p.I + d.row0;
                     ok = issue(d, wm + r * rb_ug, static_cast<uint32_t>(kStageRows * rb_ug), sm + r,
                                kStageRows * 4);
@@ -430,13 +445,16 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
             rq.exit = 0;
             mbar_arrive(&s.areq_full[aslot]);
             d.aslot = aslot;
-            const int c_end = min(p.H, (j + 1) * p.dr);
-            for (int c0 = j * p.dr; c0 < c_end && ok; c0 += p.sr_down) {
-                d.row0 = c0;
-                d.nrows = min(p.sr_down, c_end - c0);
-                d.first = (c0 == j * p.dr);
-                d.last = (c0 + p.sr_down >= c_end);
-                const size_t r = static_cast<size_t>(d.e) * p.H + c0;
+            // always two stages (one per consumer group), the rows split evenly
+            const int c_beg = j * p.dr, n = min(p.H, c_beg + p.dr) - c_beg, h1 = (n + 1) / 2;
+            d.nst = kDownStagesPerTile;
+            for (int q = 0; q < kDownStagesPerTile && ok; ++q) {
+                d.sit = q;
+                d.row0 = c_beg + (q == 0 ? 0 : h1);
+                d.nrows = q == 0 ? h1 : n - h1;
+                d.first = q == 0;
+                d.last = q == kDownStagesPerTile - 1;
+                const size_t r = static_cast<size_t>(d.e) * p.H + d.row0;
                 ok = issue(d, ex.w_down + r * rb_d, static_cast<uint32_t>(d.nrows * rb_d), ex.s_down + r,
                            static_cast<uint32_t>(d.nrows * 4));
             }
@@ -452,7 +470,8 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         s.areq[aslot].exit = 1;
         mbar_arrive(&s.areq_full[aslot]);
     }
-    if (acquire_stage()) {
+    for (int g = 0; g < kGroups; ++g) {  // one end marker per consumer group
+        if (!acquire_stage()) break;
         s.desc[stage].type = D_EXIT;
         mbar_arrive(&s.full[stage]);
         advance();
@@ -571,15 +590,17 @@ __device__ void consumer_init(const FusedParams& p, const Smem& s) {
 
 // One router stage: logits of rows e0 .. e0 + nrows - 1 for every token.
 template <int NT>
-__device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int nrows, const uint8_t* sbuf) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+__device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int nrows, const uint8_t* sbuf,
+                               int g) {
+    const int gtid = threadIdx.x % kGroupThreads, gwarp = gtid >> 5, lane = gtid & 31;
     const int h4 = p.H / 4;
+    double* red = s.red + g * (kGroupWarps * kMaxRouterRows * kMaxT);
     double acc[kMaxRouterRows][NT];
 #pragma unroll
     for (int q = 0; q < kMaxRouterRows; ++q)
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[q][t] = 0.0;
-    for (int j = tid; j < h4; j += kConsumers) {
+    for (int j = gtid; j < h4; j += kGroupThreads) {
         double xv[NT][4];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -610,21 +631,22 @@ __device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int 
         for (int t = 0; t < NT; ++t) {
             if (q < nrows) {
                 const double v = warp_sum_f64(acc[q][t]);
-                if (lane == 0) s.red[(warp * kMaxRouterRows + q) * kMaxT + t] = v;
+                if (lane == 0) red[(gwarp * kMaxRouterRows + q) * kMaxT + t] = v;
             }
         }
-    consumers_sync();
-    if (tid < nrows * p.T) {
+    group_sync(g);
+    if (gtid < nrows * p.T) {
         // logit rounded once to fp32, sigmoid in fp64 rounded once; published
         // with this launch's tag in the same 64-bit word
-        const int q = tid / p.T, t = tid % p.T;
+        const int q = gtid / p.T, t = gtid % p.T;
         double sum = 0.0;
-        for (int w = 0; w < kConsumerWarps; ++w) sum += s.red[(w * kMaxRouterRows + q) * kMaxT + t];
+        for (int w = 0; w < kGroupWarps; ++w) sum += red[(w * kMaxRouterRows + q) * kMaxT + t];
         const double l = static_cast<double>(__double2float_rn(sum));
         const float sc = __double2float_rn(1.0 / (1.0 + exp(-l)));
         st_relaxed_gpu_u64(p.scores + static_cast<size_t>(t) * p.E + e0 + q,
                            (static_cast<unsigned long long>(*s.tag) << 32) | __float_as_uint(sc));
     }
+    group_sync(g);  // the reduction buffer is reused by this group's next router stage
 }
 
 // Selection and union for the whole batch, computed by all consumer threads
@@ -849,62 +871,75 @@ struct ActRegs {
 // up/gate stage, NT = 1: the token's Q8_0(x) words are in registers.
 template <int QT>
 __device__ __forceinline__ void consume_ug_reg(const FusedParams& p, const Smem& s, float* dst, int row0,
-                                               const uint8_t* sbuf, const ActRegs<kRegChunksUg>& ar) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                               const uint8_t* sbuf, const ActRegs<kRegChunksUg>& ar, int gw) {
+    const int lane = threadIdx.x & 31;
     const int nbH = p.H / 32;
     const size_t rb = static_cast<size_t>(p.H) * QT / 8;
-    const uint8_t* wrow = sbuf + warp * rb;
-    float acc = 0.0f;
+    const uint8_t* w0 = sbuf + gw * rb;                  // rows gw and gw + kGroupWarps of the stage
+    const uint8_t* w1 = sbuf + (gw + kGroupWarps) * rb;
+    float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < kRegChunksUg; ++j) {
         const int b = lane + 32 * j;
         if (b < nbH) {
-            const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
-            const int isum = block_dot<QT>(wb, ar.a0[j], ar.a1[j], s.qs[b]);
-            acc = fmaf(static_cast<float>(isum), s.qd[b], acc);
+            const WBlock<QT> wb0 = load_wblock_smem<QT>(w0, b);
+            const WBlock<QT> wb1 = load_wblock_smem<QT>(w1, b);
+            const int qs = s.qs[b];
+            const float qd = s.qd[b];
+            acc0 = fmaf(static_cast<float>(block_dot<QT>(wb0, ar.a0[j], ar.a1[j], qs)), qd, acc0);
+            acc1 = fmaf(static_cast<float>(block_dot<QT>(wb1, ar.a0[j], ar.a1[j], qs)), qd, acc1);
         }
     }
-    const float v = warp_sum_f32(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+        acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+    }
     if (lane == 0) {
         const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
-        dst[row0 % kUgTileRows + warp] = __fmul_rn(v, sc[warp]);
+        dst[row0 % kUgTileRows + gw] = __fmul_rn(acc0, sc[gw]);
+        dst[row0 % kUgTileRows + gw + kGroupWarps] = __fmul_rn(acc1, sc[gw + kGroupWarps]);
     }
 }
 
 // up/gate stage, NT > 1: activations read from the shared-memory cache.
 template <int QT, int NT>
 __device__ __forceinline__ void consume_ug_smem(const FusedParams& p, const Smem& s, const Desc& d, float* dst,
-                                                const uint8_t* sbuf) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                                const uint8_t* sbuf, int gw) {
+    const int lane = threadIdx.x & 31;
     const int nbH = p.H / 32;
     const size_t rb = static_cast<size_t>(p.H) * QT / 8;
-    const uint8_t* wrow = sbuf + warp * rb;
     const int n_tok = d.n_tok;
     int tok[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) tok[t] = t < n_tok ? d.tok[t] : 0;
-    float acc[NT];
+    const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {  // rows gw and gw + kGroupWarps of the stage
+        const int rs = gw + h * kGroupWarps;
+        const uint8_t* wrow = sbuf + rs * rb;
+        float acc[NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
+        for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
 #pragma unroll 2
-    for (int b = lane; b < nbH; b += 32) {
-        const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
+        for (int b = lane; b < nbH; b += 32) {
+            const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (t < n_tok) {
+                    const int q = tok[t] * nbH + b;
+                    const int isum = block_dot<QT>(wb, s.q0[q], s.q1[q], s.qs[q]);
+                    acc[t] = fmaf(static_cast<float>(isum), s.qd[q], acc[t]);
+                }
+            }
+        }
+        const int r = d.row0 % kUgTileRows + rs;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             if (t < n_tok) {
-                const int q = tok[t] * nbH + b;
-                const int isum = block_dot<QT>(wb, s.q0[q], s.q1[q], s.qs[q]);
-                acc[t] = fmaf(static_cast<float>(isum), s.qd[q], acc[t]);
+                const float v = warp_sum_f32(acc[t]);
+                if (lane == 0) dst[t * kUgTileRows + r] = __fmul_rn(v, sc[rs]);
             }
-        }
-    }
-    const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
-    const int r = d.row0 % kUgTileRows + warp;
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        if (t < n_tok) {
-            const float v = warp_sum_f32(acc[t]);
-            if (lane == 0) dst[t * kUgTileRows + r] = __fmul_rn(v, sc[warp]);
         }
     }
 }
@@ -913,8 +948,8 @@ __device__ __forceinline__ void consume_ug_smem(const FusedParams& p, const Smem
 template <int QT>
 __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0, int nrows, int pair,
                                                  const uint8_t* sbuf, const ActRegs<kRegChunksDown>& ar,
-                                                 const float* ad, const int32_t* as) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                                 const float* ad, const int32_t* as, int gw) {
+    const int lane = threadIdx.x & 31;
     const int nbI = p.I / 32;
     const size_t rb = static_cast<size_t>(p.I) * QT / 8;
     const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
@@ -922,7 +957,7 @@ __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0,
 #pragma unroll
     for (int k = 0; k < kMaxDownRowsPerWarp; ++k) {
         acc[k] = 0.0f;
-        const int r = warp + kConsumerWarps * k;
+        const int r = gw + kGroupWarps * k;
         if (r < nrows) {
             const uint8_t* wrow = sbuf + r * rb;
 #pragma unroll
@@ -938,7 +973,7 @@ __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0,
     }
 #pragma unroll
     for (int k = 0; k < kMaxDownRowsPerWarp; ++k) {
-        const int r = warp + kConsumerWarps * k;
+        const int r = gw + kGroupWarps * k;
         if (r < nrows) {
             const float v = warp_sum_f32(acc[k]);
             if (lane == 0) p.y[static_cast<size_t>(pair) * p.H + row0 + r] = __fmul_rn(v, sc[r]);
@@ -949,8 +984,8 @@ __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0,
 // down stage, NT > 1: activations read from the tile's shared-memory slot.
 template <int QT, int NT>
 __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Smem& s, const Desc& d,
-                                                  const uint8_t* sbuf) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                                                  const uint8_t* sbuf, int gw) {
+    const int lane = threadIdx.x & 31;
     const int nbI = p.I / 32;
     const size_t rb = static_cast<size_t>(p.I) * QT / 8;
     const uint8_t* act = s.act + static_cast<size_t>(d.aslot) * p.act_bytes;
@@ -959,7 +994,7 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
     int pair[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) pair[t] = d.pair[t];
-    for (int r = warp; r < nrows; r += kConsumerWarps) {
+    for (int r = gw; r < nrows; r += kGroupWarps) {
         const uint8_t* wrow = sbuf + r * rb;
         float acc[NT];
 #pragma unroll
@@ -990,9 +1025,10 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
 }
 
 // Hands a finished tile (or the end) to epilogue warp tb through task slot tb.
-__device__ __forceinline__ void push_task(const Smem& s, int tb, const Desc* d, int type) {
-    const int tid = threadIdx.x, lane = tid & 31;
-    if (tid == 0) {
+// Every consumer warp arrives once per tile; `writer` (one warp) fills the task first.
+__device__ __forceinline__ void push_task(const Smem& s, int tb, const Desc* d, int type, bool writer) {
+    const int lane = threadIdx.x & 31;
+    if (writer && lane == 0) {
         Task& tk = s.task[tb];
         tk.type = type;
         if (d) {
@@ -1010,10 +1046,12 @@ __device__ __forceinline__ void push_task(const Smem& s, int tb, const Desc* d, 
 
 template <int QT, int NT>
 __device__ void consumer(const FusedParams& p, const Smem& s) {
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = warp / kGroupWarps, gw = warp % kGroupWarps;
     const size_t slot_bytes = static_cast<size_t>(p.stage_bytes) + kScaleBytes;
     consumer_init(p, s);
-    int stage = 0, aslot = 0, tb = 0;
+    // group g takes ring stages g, g + kGroups, g + 2 kGroups, ...
+    int stage = g, aslot = 0, tb = 0;
     uint32_t phase = 0, aphase = 0;
     uint32_t tph[kTaskSlots] = {0, 0};
     // Waits for the current stage; returns its type (D_EXIT on timeout).
@@ -1027,8 +1065,9 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     auto release = [&]() {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.empty[stage]);
-        if (++stage == p.nstage) {
-            stage = 0;
+        stage += kGroups;
+        if (stage >= p.nstage) {
+            stage -= p.nstage;
             phase ^= 1u;
         }
     };
@@ -1048,13 +1087,16 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     // phase A: router rows (the helper warp routes meanwhile), then Q8_0 of x
     while (type == D_ROUTER) {
         const int e0 = s.desc[stage].e, nrows = s.desc[stage].nrows;
-        consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes);
+        consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes, g);
         release();
         type = next_type();
     }
     quantize_x<QT>(p, s);
     consumers_sync();
-    // phases B and C: runs of up/gate tiles and of down tiles, interleaved
+    // phases B and C: runs of up/gate tiles and of down tiles.  A tile's
+    // stages alternate between the groups, so every warp sees every tile:
+    // its first stage of a tile (sit < kGroups) claims the task slot or the
+    // activation records, its last one (sit + kGroups >= nst) hands the tile on.
     bool ok = true;
     while (ok && (type == D_UG || type == D_DOWN)) {
         if (type == D_UG) {
@@ -1072,18 +1114,18 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
             while (type == D_UG) {
                 const Desc& d = s.desc[stage];
                 const uint8_t* sbuf = s.ring + stage * slot_bytes;
-                if (d.first && !task_slot_free()) {
+                if (d.sit < kGroups && !task_slot_free()) {
                     ok = false;
                     break;
                 }
                 float* dst = (d.mat == 0 ? s.gbuf : s.ubuf) + tb * kMaxT * kUgTileRows;
                 if constexpr (NT == 1) {
-                    consume_ug_reg<QT>(p, s, dst, d.row0, sbuf, ar);
+                    consume_ug_reg<QT>(p, s, dst, d.row0, sbuf, ar, gw);
                 } else {
-                    consume_ug_smem<QT, NT>(p, s, d, dst, sbuf);
+                    consume_ug_smem<QT, NT>(p, s, d, dst, sbuf, gw);
                 }
-                if (d.last) {
-                    push_task(s, tb, &d, D_UG);
+                if (d.sit + kGroups >= d.nst) {
+                    push_task(s, tb, &d, D_UG, d.sit == d.nst - 1 && gw == 0);
                     next_task();
                 }
                 release();
@@ -1096,7 +1138,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
             while (type == D_DOWN) {
                 const Desc& d = s.desc[stage];
                 const uint8_t* sbuf = s.ring + stage * slot_bytes;
-                if (d.first) {
+                if (d.sit < kGroups) {
                     if (!mbar_wait(&s.afull[aslot], aphase, kConsumerWait)) {
                         record_status(p.status, MOE_EDEVICE_TIMEOUT);
                         ok = false;
@@ -1117,11 +1159,11 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                     }
                 }
                 if constexpr (NT == 1) {
-                    consume_down_reg<QT>(p, d.row0, d.nrows, d.pair[0], sbuf, ar, ad, as);
+                    consume_down_reg<QT>(p, d.row0, d.nrows, d.pair[0], sbuf, ar, ad, as, gw);
                 } else {
-                    consume_down_smem<QT, NT>(p, s, d, sbuf);
+                    consume_down_smem<QT, NT>(p, s, d, sbuf, gw);
                 }
-                if (d.last) {
+                if (d.sit + kGroups >= d.nst) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.aempty[aslot]);
                     if (++aslot == kActSlots) {
@@ -1132,7 +1174,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                         ok = false;
                         break;
                     }
-                    push_task(s, tb, &d, D_DOWN);
+                    push_task(s, tb, &d, D_DOWN, d.sit == d.nst - 1 && gw == 0);
                     next_task();
                 }
                 release();
@@ -1143,7 +1185,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     // hand the end to both epilogue warps
     for (int i = 0; i < kTaskSlots; ++i) {
         if (!task_slot_free()) break;
-        push_task(s, tb, nullptr, D_EXIT);
+        push_task(s, tb, nullptr, D_EXIT, warp == 0);
         next_task();
     }
 }
@@ -1273,7 +1315,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
     if (tid == 0) {
         for (int i = 0; i < p.nstage; ++i) {
             mbar_init(&s.full[i], 1);
-            mbar_init(&s.empty[i], kConsumerWarps);
+            mbar_init(&s.empty[i], kGroupWarps);
         }
         for (int i = 0; i < kActSlots; ++i) {
             mbar_init(&s.afull[i], 1);
@@ -1334,7 +1376,7 @@ bool fused_geometry(FusedParams& p, int qtype) {
     size_t stage = std::max(static_cast<size_t>(4) * p.H, kStageRows * rb_ug);
     stage = (stage + 127) / 128 * 128;
     const int sr = static_cast<int>(stage / (kStageRows * rb_d)) * kStageRows;
-    if (sr < kStageRows || sr > kConsumerWarps * kMaxDownRowsPerWarp || sr * 4 > kScaleBytes) return false;
+    if (sr < kStageRows || sr > kGroupWarps * kMaxDownRowsPerWarp || sr * 4 > kScaleBytes) return false;
     p.stage_bytes = static_cast<int>(stage);
     p.rps = std::min<int>(kMaxRouterRows, static_cast<int>(stage / (4 * static_cast<size_t>(p.H))));
     p.n_rt = (p.E + p.rps - 1) / p.rps;
