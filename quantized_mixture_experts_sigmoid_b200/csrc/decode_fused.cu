@@ -86,6 +86,7 @@ constexpr long kProducerWait = 1L << 22;
 constexpr long kConsumerWait = 1L << 24;
 constexpr long kEpilogueWait = 1L << 25;
 constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps (group g: 2 + g)
+constexpr int kBarAfterDep = 4;      // all warps but the producer, after the grid dependency
 static_assert(kStageRows == 2 * kGroupWarps, "an up/gate stage gives each warp of a group two rows");
 static_assert(kDownStagesPerTile == kGroups && (2 * (kUgTileRows / kStageRows)) % kGroups == 0,
               "the stages of every tile reach every consumer group");
@@ -355,12 +356,20 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         return true;
     };
 
-    // the first ticket of CTA b is b (no round trip before the first copy);
-    // later ones come from the shared counter
+    // The first ticket of CTA b is b: no round trip before the first copy,
+    // and none of the workspace is touched, so it streams while the previous
+    // grid in the stream finishes.  Later tickets come from the shared
+    // counter, claimed once that grid has completed.
     int next = blockIdx.x;
+    bool dep_done = false;
     while (ok) {
+        if (next < 0) {
+            grid_dependency_wait();
+            dep_done = true;
+            next = static_cast<int>(gridDim.x) + atomicAdd(&p.sync->ticket, 1);
+        }
         const int cur = next;
-        next = static_cast<int>(gridDim.x) + atomicAdd(&p.sync->ticket, 1);
+        next = dep_done ? static_cast<int>(gridDim.x) + atomicAdd(&p.sync->ticket, 1) : -1;
         Desc d{};
         if (cur < nrt) {  // router rows e0 .. e0 + n - 1
             d.type = D_ROUTER;
@@ -1331,9 +1340,16 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.areq_free[i], 1);
         }
         fence_mbar_init();
-        *s.tag = static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch))) + 1u;
+        grid_launch_dependents();
     }
     __syncthreads();
+    // everyone but the producer waits for the previous grid here (x, the
+    // workspace and its launch counter may come from it)
+    if (warp != kProducerWarp) {
+        grid_dependency_wait();
+        if (tid == 0) *s.tag = static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch))) + 1u;
+        named_bar_sync(kBarAfterDep, kThreadsF - 32);
+    }
     if (warp == kProducerWarp) {
         if (lane == 0) producer<QT>(p, s);
     } else if (warp == kHelperWarp) {
@@ -1418,8 +1434,20 @@ cudaError_t launch_decode_fused(const FusedParams& p, cudaStream_t st) {
     }
     e = ensure_smem(kern, smem);
     if (e != cudaSuccess) return e;
+    // programmatic dependent launch: this grid may start while the previous
+    // one in the stream drains (it waits for it before touching shared data)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreadsF);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     void* args[] = {const_cast<FusedParams*>(&p)};
-    e = cudaLaunchKernel(kern, dim3(grid), dim3(kThreadsF), args, smem, st);
+    e = cudaLaunchKernelExC(&cfg, kern, args);
     if (e != cudaSuccess) return e;
     return counted(cudaGetLastError());
 }

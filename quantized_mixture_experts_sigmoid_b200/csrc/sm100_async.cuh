@@ -114,6 +114,13 @@ __device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long* p, unsign
     asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Programmatic dependent launch: let the next grid in the stream start launching
+// (its CTAs become resident as this grid's CTAs exit) / wait until the previous
+// grid has completed and its memory is visible.  Both are no-ops without a
+// programmatic launch dependency.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // Fire-and-forget add with release semantics (orders this thread's earlier writes before it).
