@@ -245,6 +245,23 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
                       float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Which kernels moe_layer_forward runs for these shapes (host-only query, no
+ * launch; this library's own introspection, not a step of the pages' layer):
+ *   MOE_PATH_FUSED        one persistent launch for the whole layer (T <= 4,
+ *                         T*top_k <= 32, n_expert <= 256 and a multiple of 32,
+ *                         groups of a multiple of 32 experts, fits shared memory);
+ *   MOE_PATH_TENSOR_CORE  batch-union FFN on tcgen05 tensor cores (T > 4, int4,
+ *                         hidden and inter multiples of 64, shared expert shaped
+ *                         like the routed ones);
+ *   MOE_PATH_GENERAL      router, union, Q8_0, integer-dot expert kernels, combine.
+ * Returns one of those or MOE_EINVAL.
+ */
+#define MOE_PATH_FUSED 1
+#define MOE_PATH_TENSOR_CORE 2
+#define MOE_PATH_GENERAL 3
+int moe_layer_path(int T, const moe_router_cfg* cfg, const moe_experts* routed, const moe_experts* shared);
+
+/*
  * Read (and clear when `clear` != 0) the device status word that kernels of
  * moe_layer_forward / moe_expert_ffn_q record in `ws`.  Synchronises `stream`.
  * *status receives MOE_OK or the first device-side MOE_E* code.  A clear also

@@ -311,7 +311,9 @@ static int row_bytes(int qtype, int n) { return n * qtype / 8; }
 /*
  * One expert on one token: Q8_0(x) -> gate and up rows -> SwiGLU ->
  * Q8_0(h) -> down rows.  The SwiGLU is h = silu(g) * u with
- * silu(g) = g / (1 + e^-g) in fp32, as in GLM-5.2's expert MLP; h is
+ * silu(g) = g / (1 + e^-g), as in GLM-5.2's expert MLP, evaluated in fp64 and
+ * rounded once to fp32 (the router's sigmoid is evaluated the same way), then
+ * multiplied by u in fp32; h is
  * re-quantised to Q8_0 because the integer-dot kernel runs against Q8_0
  * activations ([HN] "구현된 주요 기능").  The shared expert uses the same
  * function ([HN] router bullet lists the shared expert; [MO] "3단계 메모리
@@ -343,7 +345,7 @@ int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* 
             const float g = oracle_qdot(codes, ex->s_gate[e][r], qa, da, H);
             oracle_unpack(ex->w_up[e] + (size_t)r * rb_in, q, H, codes);
             const float u = oracle_qdot(codes, ex->s_up[e][r], qa, da, H);
-            const float silu = g / (1.0f + expf(-g));
+            const float silu = (float)((double)g / (1.0 + exp(-(double)g)));
             h[r] = silu * u;
         }
 #pragma omp single

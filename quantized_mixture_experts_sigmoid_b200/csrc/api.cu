@@ -105,6 +105,10 @@ struct LayerWs {
     float* dhs;
     float* y;
     float* ys;
+    // tensor-core batch-union path (T > kFusedMaxTokens, int4)
+    __half* xc;    // Q8_0(x) codes as fp16 [T][H]
+    __half* hc;    // Q8_0(h) codes as fp16 [(P + T)][I]
+    float* hs;     // their block scales
     // fused small-batch path only (T <= kFusedMaxTokens)
     int32_t* pair_of;
     uint8_t* qrec;
@@ -137,6 +141,12 @@ LayerWs carve_layer(void* ws, int T, const moe_router_cfg& c, const moe_experts&
         L.ys = cv.take<float>(static_cast<size_t>(T) * H);
     }
     L.y = cv.take<float>(P * H);
+    if (T > kFusedMaxTokens && tc_gemm_supported(r, s, c.n_expert)) {
+        const size_t rows = P + static_cast<size_t>(T);
+        L.xc = cv.take<__half>(static_cast<size_t>(T) * H);
+        L.hc = cv.take<__half>(rows * I);
+        L.hs = cv.take<float>(rows * I / 32);
+    }
     if (T <= kFusedMaxTokens) {
         L.pair_of = cv.take<int32_t>(P);
         L.qrec = cv.take<uint8_t>((P + T) * fused_record_bytes(I));
@@ -375,6 +385,59 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
                                    L.pair_slot, nullptr, L.status, st))))
         return rc;
     if ((rc = cuda_rc(launch_q8_0(x, true, T, H, L.qx, L.dx, st)))) return rc;
+
+    if (L.xc) {  // many tokens per expert: tensor-core batch-union FFN
+        const int I = routed->inter, P = T * K;
+        if ((rc = cuda_rc(launch_codes_f16(L.qx, static_cast<size_t>(T) * H, L.xc, st)))) return rc;
+        GemmParams gp{};
+        gp.T = T;
+        gp.H = H;
+        gp.I = I;
+        gp.P = P;
+        gp.K = K;
+        gp.has_shared = shared != nullptr;
+        gp.n_unique = L.n_unique;
+        gp.uniq = L.uniq;
+        gp.offsets = L.offsets;
+        gp.pair_tok = L.pair_tok;
+        gp.pair_slot = L.pair_slot;
+        gp.status = L.status;
+        GemmOperands go{};
+        go.n_expert = E;
+        // up/gate: Q8_0(h) per pair (union order), shared rows last
+        gp.a_codes = L.xc;
+        gp.a_scales = L.dx;
+        gp.s_a = routed->s_gate;
+        gp.s_b = routed->s_up;
+        gp.s_a_sh = shared ? shared->s_gate : nullptr;
+        gp.s_b_sh = shared ? shared->s_up : nullptr;
+        gp.h_codes = L.hc;
+        gp.h_scales = L.hs;
+        go.w0 = routed->w_gate;
+        go.w1 = routed->w_up;
+        go.w0s = shared ? shared->w_gate : nullptr;
+        go.w1s = shared ? shared->w_up : nullptr;
+        const bool timed = g_prof.begin(st);
+        rc = cuda_rc(launch_moe_gemm(kGemmUpGate, gp, go, st));
+        if (timed) g_prof.end(st);
+        if (rc) return rc;
+        // down: fp32 output per (token, slot), shared rows separately
+        gp.a_codes = L.hc;
+        gp.a_scales = L.hs;
+        gp.s_a = routed->s_down;
+        gp.s_b = nullptr;
+        gp.s_a_sh = shared ? shared->s_down : nullptr;
+        gp.s_b_sh = nullptr;
+        gp.y = L.y;
+        gp.ys = shared ? L.ys : nullptr;
+        go.w0 = routed->w_down;
+        go.w1 = nullptr;
+        go.w0s = shared ? shared->w_down : nullptr;
+        go.w1s = nullptr;
+        if ((rc = cuda_rc(launch_moe_gemm(kGemmDown, gp, go, st)))) return rc;
+        return cuda_rc(launch_combine(L.y, w, shared ? L.ys : nullptr, T, K, H, out, out_dtype, st));
+    }
+
     const UnionView un{L.n_unique, L.uniq, L.offsets, L.pair_tok, L.pair_slot,
                        static_cast<int>(std::min<long long>(E, static_cast<long long>(T) * K))};
     const bool timed = g_prof.begin(st);
@@ -388,6 +451,20 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
     if (shared && (rc = cuda_rc(launch_expert_down(*shared, L.qhs, L.dhs, T, 1, dense, L.ys, st))))
         return rc;
     return cuda_rc(launch_combine(L.y, w, shared ? L.ys : nullptr, T, K, H, out, out_dtype, st));
+}
+
+int moe_layer_path(int T, const moe_router_cfg* cfg, const moe_experts* routed, const moe_experts* shared) {
+    if (!cfg || !routed || T <= 0 || check_cfg(cfg) || check_experts(routed) || (shared && check_experts(shared)))
+        return MOE_EINVAL;
+    const LayerWs L = carve_layer(nullptr, T, *cfg, *routed, shared);
+    FusedParams f;
+    void* fake = reinterpret_cast<void*>(static_cast<uintptr_t>(4096));  // geometry only: nothing is dereferenced
+    const uint16_t* fx = reinterpret_cast<const uint16_t*>(fake);
+    if (fused_params(f, L, fake, fx, T, reinterpret_cast<const float*>(fake), reinterpret_cast<const float*>(fake),
+                     *cfg, *routed, shared, fake, MOE_OUT_F32, nullptr, nullptr))
+        return MOE_PATH_FUSED;
+    if (T > kFusedMaxTokens && tc_gemm_supported(*routed, shared, cfg->n_expert)) return MOE_PATH_TENSOR_CORE;
+    return MOE_PATH_GENERAL;
 }
 
 int moe_profile_enable(int on) {

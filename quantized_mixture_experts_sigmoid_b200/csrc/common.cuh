@@ -74,10 +74,12 @@ __device__ __forceinline__ int8_t q8_0_lane(float v, float* d_out) {
     return static_cast<int8_t>(r);
 }
 
-// silu(g) * u with the same operation order as the definition: g / (1 + e^-g), then * u.
+// silu(g) * u: silu(g) = g / (1 + e^-g) evaluated in fp64 and rounded once to
+// fp32 (as the router's sigmoid), then times u in fp32.
 __device__ __forceinline__ float swiglu(float g, float u) {
-    const float den = __fadd_rn(1.0f, expf(-g));
-    return __fmul_rn(__fdiv_rn(g, den), u);
+    const double dg = static_cast<double>(g);
+    const float silu = __double2float_rn(__ddiv_rn(dg, __dadd_rn(1.0, exp(-dg))));
+    return __fmul_rn(silu, u);
 }
 
 __device__ __forceinline__ void record_status(int32_t* status, int code) {

@@ -1,6 +1,8 @@
 // Launch wrappers of the library's kernels (internal; the C ABI is in moe.h).
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -112,6 +114,42 @@ struct FusedParams {
 // Bytes of one pair's Q8_0(h) record: two 16-byte planes per block, the block
 // scales and block sums, padded so records can be bulk-copied back to back.
 inline size_t fused_record_bytes(int I) { return (static_cast<size_t>(I) + I / 4 + 15) & ~size_t(15); }
+
+// ------------------------------------------------------------ tensor-core batch-union FFN
+// (prefill and long verify: every unique expert applied to its tokens in 128-row tiles)
+constexpr int kGemmUpGate = 0, kGemmDown = 1;
+
+struct GemmParams {
+    int T, H, I, P, K, has_shared;
+    const int32_t* n_unique;
+    const int32_t* uniq;
+    const int32_t* offsets;
+    const int32_t* pair_tok;
+    const int32_t* pair_slot;
+    const void* a_codes;     // activation Q8_0 codes as fp16: up/gate x [T][H]; down h [(P + T)][I]
+    const float* a_scales;   // their block scales [rows][K / 32]
+    const float* s_a;        // row scales: up/gate: gate [E][I]; down: down [E][H]
+    const float* s_b;        // up/gate: up [E][I]
+    const float* s_a_sh;     // shared expert's
+    const float* s_b_sh;
+    void* h_codes;           // up/gate out: Q8_0(h) codes as fp16 [(P + T)][I] (union order, shared rows last)
+    float* h_scales;         //              block scales [(P + T)][I / 32]
+    float* y;                // down out: routed [T][K][H]
+    float* ys;               //           shared [T][H]
+    int32_t* status;
+};
+
+struct GemmOperands {
+    const void* w0;          // packed routed weights: gate (up/gate) or down
+    const void* w1;          // packed routed up weights
+    const void* w0s;         // shared expert's
+    const void* w1s;
+    int n_expert;
+};
+
+bool tc_gemm_supported(const moe_experts& r, const moe_experts* s, int E);
+cudaError_t launch_codes_f16(const int8_t* q, size_t n, __half* out, cudaStream_t st);
+cudaError_t launch_moe_gemm(int mode, const GemmParams& p, const GemmOperands& o, cudaStream_t st);
 
 // Fills the geometry fields; false if the fused kernel cannot take this shape.
 bool fused_geometry(FusedParams& p, int qtype);

@@ -88,7 +88,7 @@ EXPORTS = ["moe_strerror", "moe_route_workspace_bytes", "moe_route", "moe_union"
            "moe_quantize_q8_0", "moe_expert_ffn_workspace_bytes", "moe_expert_ffn_q",
            "moe_combine", "moe_layer_workspace_bytes", "moe_layer_forward",
            "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count",
-           "moe_route_noalloc"]
+           "moe_route_noalloc", "moe_layer_path"]
 
 
 def lib() -> ctypes.CDLL:
@@ -115,6 +115,8 @@ def lib() -> ctypes.CDLL:
     L.moe_combine.argtypes = [vp, vp, vp, i, i, i, vp, i, vp]
     L.moe_layer_workspace_bytes.argtypes = [i, vp, vp, vp]
     L.moe_layer_workspace_bytes.restype = sz
+    L.moe_layer_path.argtypes = [i, vp, vp, vp]
+    L.moe_layer_path.restype = i
     L.moe_layer_forward.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.moe_workspace_status.argtypes = [vp, i, vp, vp]
     L.moe_profile_enable.argtypes = [i]
@@ -212,6 +214,19 @@ def moe_layer_workspace_bytes(T: int, cfg: RouterCfg, routed: ExpertSet, shared:
     ss = shared.struct() if shared is not None else None
     return lib().moe_layer_workspace_bytes(T, ctypes.byref(cfg), ctypes.byref(rs),
                                            ctypes.byref(ss) if ss is not None else None)
+
+
+PATH_FUSED, PATH_TENSOR_CORE, PATH_GENERAL = 1, 2, 3
+
+
+def moe_layer_path(T: int, cfg: RouterCfg, routed: ExpertSet, shared: ExpertSet | None) -> int:
+    """Which kernels moe_layer_forward runs for these shapes (PATH_*)."""
+    rs = routed.struct()
+    ss = shared.struct() if shared is not None else None
+    rc = lib().moe_layer_path(T, ctypes.byref(cfg), ctypes.byref(rs), ctypes.byref(ss) if ss is not None else None)
+    if rc < 0:
+        raise MoeError("moe_layer_path", rc)
+    return rc
 
 
 def moe_layer_forward(x, w_router, bias, cfg: RouterCfg, routed: ExpertSet,

@@ -119,3 +119,21 @@ def test_workspace_sizes_cover_the_buffers():
     assert b1 % 256 == 0 and b2048 > b1
     # at least the per-pair fp32 outputs, the routed and shared h codes and the logits
     assert b2048 >= 2048 * 8 * 6144 * 4 + 2048 * 9 * 2048 + 2048 * 256 * 4
+
+
+def test_layer_path_query():
+    # host-only: which kernels a call would run (nothing is launched)
+    L = moe.lib()
+    glm = _cfg()
+    r, s = _ex(), _ex(n=1)
+    path = lambda T, cfg=glm, rr=r, ss=s: L.moe_layer_path(T, ctypes.byref(cfg), ctypes.byref(rr),
+                                                          ctypes.byref(ss) if ss is not None else None)
+    assert path(1) == moe.PATH_FUSED
+    assert path(4) == moe.PATH_FUSED
+    assert path(5) == moe.PATH_TENSOR_CORE
+    assert path(2048) == moe.PATH_TENSOR_CORE
+    assert path(2048, rr=_ex(q=8)) == moe.PATH_GENERAL           # int8 experts: integer-dot kernels
+    assert path(2048, rr=_ex(H=544, I=288), ss=_ex(n=1, H=544, I=288)) == moe.PATH_GENERAL  # K not a multiple of 64
+    small = _cfg(E=16, G=4, TG=2, K=2)
+    assert path(4, cfg=small, rr=_ex(n=16)) == moe.PATH_GENERAL  # groups of 4 experts: no fused kernel
+    assert path(0) == moe.MOE_EINVAL

@@ -37,13 +37,17 @@ SHAPES = {
                                           topk_group=2, top_k=6, qtype=2),
     "fused_ragged_int8": synth.LayerShape("fused_ragged_int8", T=4, H=544, I=288, E=96, n_group=3,
                                           topk_group=2, top_k=5, qtype=8),
+    # many tokens per expert on the tensor cores: several 128-row tiles per
+    # expert, ragged N and K tails (I = 192, H = 320), shared expert included
+    "tc_small": synth.LayerShape("tc_small", T=40, H=256, I=128, E=16, n_group=4, topk_group=2, top_k=4),
+    "tc_ragged": synth.LayerShape("tc_ragged", T=300, H=320, I=192, E=32, n_group=4, topk_group=2, top_k=6),
     "decode": synth.CONFIGS["decode"],
     "verify": synth.CONFIGS["verify"],
     "verify_int8": synth.CONFIGS["verify_int8"],
     "decode_int2": synth.CONFIGS["decode"].with_(qtype=2, name="decode_int2"),
 }
 SMALL = ["tiny", "ragged", "crowded", "crowded_int8", "crowded_int2", "fused_ragged",
-         "fused_ragged_int2", "fused_ragged_int8"]
+         "fused_ragged_int2", "fused_ragged_int8", "tc_small", "tc_ragged"]
 FULL = ["decode", "verify", "verify_int8", "decode_int2"]
 
 _cache = {}
@@ -278,14 +282,28 @@ def test_union_path_equals_per_token_path_on_gpu():
         assert np.array_equal(of_one.view(np.uint32), of_batch[t:t + 1].view(np.uint32))
 
 
+def test_union_path_equals_sub_batches_on_tensor_cores():
+    # the same property on the tensor-core path: a token's output from a batch
+    # of 300 equals its output from a batch of 5 (both above the fused size)
+    sh, dev = layer("tc_ragged")
+    x, W, b = layer_inputs(sh)
+    of_batch, _, _, _ = run_layer(sh, dev, x)
+    for t in (0, 17, 295):
+        of_sub, _, _, _ = run_layer(sh, dev, x[t:t + 5])
+        assert np.array_equal(of_sub.view(np.uint32), of_batch[t:t + 5].view(np.uint32))
+
+
 FUSED = ["fused_ragged", "fused_ragged_int2", "fused_ragged_int8", "decode", "verify", "decode_int2"]
+TENSOR_CORE = ["tc_small", "tc_ragged"]
 
 
-@pytest.mark.parametrize("name", FUSED + ["tiny", "ragged"])
+@pytest.mark.parametrize("name", FUSED + TENSOR_CORE + ["tiny", "ragged", "crowded_int8"])
 def test_layer_forward_path(name):
     # small batches with groups of a multiple of 32 experts run as one fused
-    # launch; other shapes take the multi-kernel path
+    # launch; int4 batches of more tokens on the tensor cores; other shapes take
+    # the multi-kernel integer-dot path
     sh, dev = layer(name)
+    path = moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"])
     x, W, b = layer_inputs(sh)
     xd = to_dev_bf16(x)
     ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
@@ -296,9 +314,11 @@ def test_layer_forward_path(name):
     n = moe.lib().moe_launch_count() - n0
     assert moe.moe_workspace_status(ws) == 0
     if name in FUSED:
-        assert n == 1
+        assert path == moe.PATH_FUSED and n == 1
+    elif name in TENSOR_CORE:
+        assert path == moe.PATH_TENSOR_CORE and n > 1
     else:
-        assert n > 1
+        assert path == moe.PATH_GENERAL and n > 1
 
 
 def test_layer_forward_repeated_calls_reuse_workspace():
