@@ -289,8 +289,9 @@ int oracle_unpack(const uint8_t* packed, int qtype, int n, int8_t* codes) {
 
 /*
  * One quantised row dot product: integer dot per 32-block, promoted with the
- * activation block's scale and summed in fp32 over blocks in ascending order,
- * then times the row scale.  [HN] "구현된 주요 기능" (integer-dot kernel with
+ * activation block's scale and accumulated in fp32 over blocks in ascending
+ * order with one fused multiply-add per block (one rounding), then times the
+ * row scale.  [HN] "구현된 주요 기능" (integer-dot kernel with
  * Q8_0 activations; per-row scales, dequant on use).
  */
 float oracle_qdot(const int8_t* wcodes, float w_scale, const int8_t* qa, const float* da, int n) {
@@ -298,8 +299,7 @@ float oracle_qdot(const int8_t* wcodes, float w_scale, const int8_t* qa, const f
     for (int b = 0; b < n / 32; ++b) {
         int32_t isum = 0;
         for (int i = 32 * b; i < 32 * b + 32; ++i) isum += (int32_t)qa[i] * (int32_t)wcodes[i];
-        const float p = (float)isum * da[b];
-        acc = acc + p;
+        acc = fmaf((float)isum, da[b], acc);  /* one rounding per block */
     }
     return acc * w_scale;
 }

@@ -8,14 +8,14 @@
 //
 // Arithmetic, exactly the quantised dot's: for every 32-block b the integer
 // dot isum_b of the activation codes with the weight codes, then
-// acc = acc + isum_b * d_b in ascending b (fp32, the multiply and the add each
-// rounded), then times the row scale.  The tensor cores produce the isum_b:
+// acc = fma(isum_b, d_b, acc) in ascending b (fp32, one rounding per block),
+// then times the row scale.  The tensor cores produce the isum_b:
 // both operands are the integer codes written as fp16 (exact: |q| <= 127 and
 // the int4 weight codes), one 32-element block per pair of K = 16 MMAs; the
 // fp32 accumulator of a block holds an integer below 2^15 (exact).  Each
 // block's result lands in its own slot of a 4-slot TMEM ring; the epilogue
 // warps fold it into per-thread fp32 accumulators in block order (packed
-// f32x2 multiply and add).  Up/gate then applies SwiGLU and Q8_0 to h (the
+// f32x2 fused multiply-add).  Up/gate then applies SwiGLU and Q8_0 to h (the
 // codes written as fp16 for the down GEMM); down writes the fp32 output per
 // (token, slot).  The result is the same, bit for bit, as the reference
 // arithmetic.
@@ -135,18 +135,14 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
     return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
 
-// acc = acc + v * d for a pair of lanes (the multiply and the add each rounded,
-// as the quantised dot's block sum orders them).
+// acc = fma(v, d, acc) for a pair of lanes: the quantised dot's block step
+// (one rounding), as a packed f32x2 fused multiply-add.
 __device__ __forceinline__ void fold2(float2& acc, uint32_t v0, uint32_t v1, float d) {
     float2 v = make_float2(__uint_as_float(v0), __uint_as_float(v1));
     float2 dd = make_float2(d, d);
-    float2 prod;
-    asm volatile("mul.rn.f32x2 %0, %1, %2;"
-                 : "=l"(reinterpret_cast<uint64_t&>(prod))
+    asm volatile("fma.rn.f32x2 %0, %1, %2, %0;"
+                 : "+l"(reinterpret_cast<uint64_t&>(acc))
                  : "l"(reinterpret_cast<uint64_t&>(v)), "l"(reinterpret_cast<uint64_t&>(dd)));
-    asm volatile("add.rn.f32x2 %0, %1, %2;"
-                 : "=l"(reinterpret_cast<uint64_t&>(acc))
-                 : "l"(reinterpret_cast<uint64_t&>(acc)), "l"(reinterpret_cast<uint64_t&>(prod)));
 }
 
 // Q8_0 of 32 values held by one thread, same arithmetic as q8_0_lane; the codes
