@@ -52,6 +52,15 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s (same nominal rate): the measured cuBLAS bf16 burst figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["bf16_tflops"]), "measured (cuBLAS bf16 burst)"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 KERNEL_SOURCES = ("decode_fused.cu", "common.cuh", "kernels.cuh", "quant.cuh", "sm100_async.cuh")
 
 
@@ -83,6 +92,13 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--pool", type=int, default=512, help="distinct seeded tokens cycled through")
+    ap.add_argument("--prefill", type=int, default=10,
+                    help="prefill layers (T = 2048) timed for the extra 'prefill' entry; 0 skips it")
+    ap.add_argument("--prefill-tokens", type=int, default=2048, help="prefill batch size (profiling: smaller)")
+    ap.add_argument("--prefill-experts", type=int, default=256,
+                    help="routed experts of the prefill layer (profiling: 32, in 4 groups)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill measurement and print its entry (for profiler captures)")
     return ap.parse_args()
 
 
@@ -181,12 +197,78 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CUDA arm
+def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
+    """The batch-union prefill layer (T = 2048, Zipf-skewed routing) on the tensor-core path:
+    whole-layer tokens/s and the two expert GEMMs' share of the dense tensor roofline."""
+    import ctypes
+
+    import torch
+    sh = synth.CONFIGS["prefill"]
+    if args.prefill_tokens != sh.T or args.prefill_experts != sh.E:
+        groups = 8 if args.prefill_experts >= 256 else 4
+        sh = sh.with_(T=args.prefill_tokens, E=args.prefill_experts, n_group=groups, topk_group=groups // 2)
+    dev = device_layer(sh)
+    x = to_dev_bf16(synth.hidden_states(sh))
+    out = torch.empty(sh.T, sh.H, dtype=torch.bfloat16, device="cuda")
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
+    path = moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"])
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+
+    for _ in range(3):
+        fwd()
+    torch.cuda.synchronize()
+    reps = max(3, args.prefill)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fwd()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    layer_ms = e0.elapsed_time(e1) / reps
+    L.moe_profile_enable(1)
+    for _ in range(reps):
+        fwd()
+    torch.cuda.synchronize()
+    kms, kn = ctypes.c_double(0), ctypes.c_int(0)
+    L.moe_profile_read(ctypes.byref(kms), ctypes.byref(kn))
+    L.moe_profile_enable(0)
+    if moe.moe_workspace_status(ws) != 0:
+        raise RuntimeError("device status error during the prefill measurement")
+    gemm_ms = kms.value / max(kn.value, 1)
+    rows = sh.T * sh.top_k + sh.T  # (token, expert) pairs plus the shared expert's rows
+    flops = 2.0 * rows * 3 * sh.H * sh.I  # up, gate and down contractions actually needed
+    peak, kind = tensor_peak()
+    achieved = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    del ws, dev
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"prefill batch-union: T={sh.T}, GLM-5.2 layer shape ({sh.E} routed experts), "
+                    "Zipf(1.1) expert popularity",
+        "path": {moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core", moe.PATH_GENERAL: "general"}[path],
+        "tokens_per_s": sh.T / (layer_ms / 1e3), "ms_per_layer": layer_ms, "layers_timed": reps,
+        "roofline": {"bound": "tensor", "kernel": "k_moe_gemm up/gate + down (both launches)",
+                     "achieved": achieved, "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
+                     "frac": achieved / peak if achieved else None, "flops_per_layer": flops,
+                     "ms_per_layer_gemms": gemm_ms,
+                     "flops_note": "2 x (T*top_k + T) x 3 x H x I: only the rows the layer needs; "
+                                   "tile padding is not counted"},
+    }
+
+
 def run_cuda(args):
     import torch
     import torch.distributed as dist
 
     from quantized_mixture_experts_sigmoid_b200 import moe
     from tests.gpu_fixtures import device_layer, to_dev_bf16
+
+    if args.prefill_only:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(prefill_measurement(args, moe, moe.lib(), device_layer, to_dev_bf16)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -282,6 +364,8 @@ def run_cuda(args):
         dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
     e2e_ms = float(t_e2e.item())
 
+    prefill = prefill_measurement(args, moe, L, device_layer, to_dev_bf16) if args.prefill else None
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -323,6 +407,8 @@ def run_cuda(args):
         "clocks": clk.summary(),
         "wall_s_timed_region": wall,
     }
+    if prefill is not None:
+        line["prefill"] = prefill
     if not args.no_cpu_baseline and world == 1:
         cb, _, _ = oracle_sample(sh, args.cpu_seconds)
         line["cpu_baseline"] = cb

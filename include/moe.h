@@ -275,9 +275,11 @@ int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream);
 /*
  * Kernel timing for benchmarks (no counterpart on the pages).  While enabled,
  * moe_layer_forward records a CUDA event pair on its stream around the
- * layer's dominant kernel (the one that streams the expert weights);
- * moe_profile_read waits for the recorded events and returns the summed
- * milliseconds and the number of timed launches since the last enable.
+ * layer's dominant work: the fused kernel (small batches), the two
+ * tensor-core expert GEMMs taken together (MOE_PATH_TENSOR_CORE), or the
+ * up/gate expert kernel (general path); moe_profile_read waits for the
+ * recorded events and returns the summed milliseconds and the number of
+ * timed regions since the last enable.
  * At most 65536 launches are timed per enable.  moe_launch_count returns the
  * number of kernels this library has launched in the process so far.
  * Host-side state; not thread-safe.

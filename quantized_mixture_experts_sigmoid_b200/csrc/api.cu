@@ -106,7 +106,7 @@ struct LayerWs {
     float* y;
     float* ys;
     // tensor-core batch-union path (T > kFusedMaxTokens, int4)
-    __half* xc;    // Q8_0(x) codes as fp16 [T][H]
+    __half* xg;    // Q8_0(x) codes as fp16 per up/gate row [(P + T)][H] (union order, shared rows last)
     __half* hc;    // Q8_0(h) codes as fp16 [(P + T)][I]
     float* hs;     // their block scales
     // fused small-batch path only (T <= kFusedMaxTokens)
@@ -143,7 +143,7 @@ LayerWs carve_layer(void* ws, int T, const moe_router_cfg& c, const moe_experts&
     L.y = cv.take<float>(P * H);
     if (T > kFusedMaxTokens && tc_gemm_supported(r, s, c.n_expert)) {
         const size_t rows = P + static_cast<size_t>(T);
-        L.xc = cv.take<__half>(static_cast<size_t>(T) * H);
+        L.xg = cv.take<__half>(rows * H);
         L.hc = cv.take<__half>(rows * I);
         L.hs = cv.take<float>(rows * I / 32);
     }
@@ -386,9 +386,9 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
         return rc;
     if ((rc = cuda_rc(launch_q8_0(x, true, T, H, L.qx, L.dx, st)))) return rc;
 
-    if (L.xc) {  // many tokens per expert: tensor-core batch-union FFN
+    if (L.xg) {  // many tokens per expert: tensor-core batch-union FFN
         const int I = routed->inter, P = T * K;
-        if ((rc = cuda_rc(launch_codes_f16(L.qx, static_cast<size_t>(T) * H, L.xc, st)))) return rc;
+        if ((rc = cuda_rc(launch_gather_codes(L.qx, H, P, P + (shared ? T : 0), L.pair_tok, L.xg, st)))) return rc;
         GemmParams gp{};
         gp.T = T;
         gp.H = H;
@@ -405,7 +405,7 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
         GemmOperands go{};
         go.n_expert = E;
         // up/gate: Q8_0(h) per pair (union order), shared rows last
-        gp.a_codes = L.xc;
+        gp.a_codes = L.xg;
         gp.a_scales = L.dx;
         gp.s_a = routed->s_gate;
         gp.s_b = routed->s_up;
@@ -417,10 +417,13 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
         go.w1 = routed->w_up;
         go.w0s = shared ? shared->w_gate : nullptr;
         go.w1s = shared ? shared->w_up : nullptr;
+        // the profiled region covers both GEMM launches (up/gate and down)
         const bool timed = g_prof.begin(st);
         rc = cuda_rc(launch_moe_gemm(kGemmUpGate, gp, go, st));
-        if (timed) g_prof.end(st);
-        if (rc) return rc;
+        if (rc) {
+            if (timed) g_prof.end(st);
+            return rc;
+        }
         // down: fp32 output per (token, slot), shared rows separately
         gp.a_codes = L.hc;
         gp.a_scales = L.hs;
@@ -434,7 +437,9 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
         go.w1 = nullptr;
         go.w0s = shared ? shared->w_down : nullptr;
         go.w1s = nullptr;
-        if ((rc = cuda_rc(launch_moe_gemm(kGemmDown, gp, go, st)))) return rc;
+        rc = cuda_rc(launch_moe_gemm(kGemmDown, gp, go, st));
+        if (timed) g_prof.end(st);
+        if (rc) return rc;
         return cuda_rc(launch_combine(L.y, w, shared ? L.ys : nullptr, T, K, H, out, out_dtype, st));
     }
 

@@ -148,7 +148,8 @@ struct GemmOperands {
 };
 
 bool tc_gemm_supported(const moe_experts& r, const moe_experts* s, int E);
-cudaError_t launch_codes_f16(const int8_t* q, size_t n, __half* out, cudaStream_t st);
+cudaError_t launch_gather_codes(const int8_t* q, int H, int P, int rows, const int32_t* pair_tok, __half* out,
+                                cudaStream_t st);
 cudaError_t launch_moe_gemm(int mode, const GemmParams& p, const GemmOperands& o, cudaStream_t st);
 
 // Fills the geometry fields; false if the fused kernel cannot take this shape.

@@ -20,14 +20,20 @@
 // (token, slot).  The result is the same, bit for bit, as the reference
 // arithmetic.
 //
+// Operand order along K.  Inside every group of 8 consecutive K positions
+// both operands hold the elements in the order 0 4 1 5 2 6 3 7: the order in
+// which the int4 conversion below produces them from one 32-bit word of packed
+// codes.  The activation rows are written in that order by k_gather_codes (x)
+// and by the up/gate epilogue (h).  A permutation inside a 32-block leaves its
+// integer dot unchanged.
+//
 // Kernel roles (one persistent CTA per SM, 16 warps):
-//   warp 0       producer: activation codes (up/gate: the tile's gathered
-//                token rows, 16-byte cp.async copies placed at their swizzled
-//                addresses; down: tensor-TMA tiles) and tensor-TMA loads of
-//                the packed weight rows;
+//   warp 0       producer: tensor-TMA tiles of the activation codes (rows in
+//                union order, contiguous) and of the packed weight rows;
 //   warp 1       MMA issuer (one lane); owns the TMEM allocation;
-//   warps 2-7    dequantise the packed int4 rows to fp16 in the swizzled
-//                operand layout;
+//   warps 2-5    dequantise the packed int4 rows to fp16 in the swizzled
+//                operand layout (one warp per SM sub-partition);
+//   warps 6-7    idle;
 //   warps 8-15   epilogue: warp 8 + h covers TMEM lanes 32 (h % 4) .. + 31 and
 //                columns 64 (h / 4) .. + 63 of each ring slot.
 // Six shared-memory stages of 64 K each.  Every wait is bounded; on timeout
@@ -48,12 +54,28 @@ constexpr int kBK = 64;             // K per stage (one 128-byte swizzle atom of
 constexpr int kStagesG = 6;
 constexpr int kRing = 4;            // TMEM slots of block results (kRing x kBN columns)
 constexpr int kThreadsG = 512;
-constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpXform0 = 2, kXformWarps = 6, kWarpEpi0 = 8, kEpiWarps = 8;
-constexpr long kGemmWait = 1L << 26;
+constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpXform0 = 2, kXformWarps = 4, kWarpEpi0 = 8, kEpiWarps = 8;
+// Register split: the CTA is launched with kLaunchRegs per thread (checked on
+// the host); warpgroups 0-1 (producer, MMA, dequantisers) lower their limit to
+// kRegsLow and the epilogue warpgroups 2-3 raise theirs to kRegsHigh, which
+// uses exactly the launched total: 2 x kRegsLow + 2 x kRegsHigh = 4 x kLaunchRegs.
+constexpr int kLaunchRegs = 128, kRegsLow = 32, kRegsHigh = 224;
+static_assert(2 * kRegsLow + 2 * kRegsHigh == 4 * kLaunchRegs, "register split must use the launched total");
+static_assert(kWarpEpi0 == 8 && kEpiWarps == 8, "epilogue = warpgroups 2 and 3");
+constexpr long kGemmWait = 1L << 26;            // polls of the final drain waits
+constexpr uint64_t kGemmWaitNs = 2000000000ull;  // pipeline waits give up after 2 s
 constexpr int kTileBytes = kBM * kBK * 2;    // one 128 x 64 fp16 operand tile (16 KiB)
 constexpr int kPackedBytes = kBN * kBK / 2;  // the stage's packed int4 weight rows (4 KiB)
 constexpr int kStageBytesG = 2 * kTileBytes + kPackedBytes;
 constexpr int kMaxItems = 1040;              // routed experts + shared expert
+constexpr int kRowClasses = kBM / 16;        // activation tiles of 16, 32, .., 128 rows
+
+// Activation-row tensor maps, one per tile height: a tile whose item has fewer
+// than 128 rows left loads only round_up(rows, 16) of them (the MMA's other
+// rows are stale and their results are discarded).
+struct RowMaps {
+    CUtensorMap m[kRowClasses];
+};
 
 struct GemmSmem {
     uint8_t* stage;       // [kStagesG][kStageBytesG], 1024-byte aligned: A | B | packed
@@ -67,8 +89,21 @@ struct GemmSmem {
     int* item_tile0;      // [kMaxItems + 1] first tile of each expert item
 };
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Pipeline wait: polls without sleeping (try_wait suspends in hardware), so a
+// phase that completes is seen at once; gives up after kGemmWaitNs.
 __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, int32_t* status) {
-    if (mbar_wait(bar, parity, kGemmWait)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255u) == 0 && globaltimer_ns() - t0 > kGemmWaitNs) break;
+    }
     record_status(status, MOE_EDEVICE_TIMEOUT);
     return false;
 }
@@ -113,20 +148,24 @@ __device__ __forceinline__ void tile_of(const GemmSmem& s, int n_items, int n_ti
 }
 
 // 8 packed int4 codes (offset binary, element 2j in the low nibble of byte j)
-// -> 8 fp16 values q = u - 8, in element order.  fp16(1024 + u) - 1032 is exact.
+// -> 8 fp16 values q = u - 8 in the order 0 4 1 5 2 6 3 7.  Masking a nibble
+// into the mantissa of fp16 1024 gives 1024 + u (low nibble of a 16-bit half)
+// or 1024 + 16 u (high nibble); 1024 + u - 1032 and (1024 + 16 u) / 16 - 72
+// are exact.
 __device__ __forceinline__ uint4 int4x8_to_f16(uint32_t w) {
-    const uint32_t bias = 0x64006400u;
-    const uint32_t p01 = ((w & 0xFu) | ((w << 12) & 0xF0000u)) | bias;
-    const uint32_t p23 = (((w >> 8) & 0xFu) | ((w << 4) & 0xF0000u)) | bias;
-    const uint32_t p45 = (((w >> 16) & 0xFu) | ((w >> 4) & 0xF0000u)) | bias;
-    const uint32_t p67 = (((w >> 24) & 0xFu) | ((w >> 12) & 0xF0000u)) | bias;
-    const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));  // 1032
+    const uint32_t ex = 0x64006400u;
+    const uint32_t e04 = (w & 0x000F000Fu) | ex, e15 = (w & 0x00F000F0u) | ex;
+    w >>= 8;
+    const uint32_t e26 = (w & 0x000F000Fu) | ex, e37 = (w & 0x00F000F0u) | ex;
+    const __half2 off = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));      // 1032
+    const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));  // 1/16
+    const __half2 m72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));        // -72
     uint4 r;
     __half2 h;
-    h = __hsub2(*reinterpret_cast<const __half2*>(&p01), off); r.x = *reinterpret_cast<uint32_t*>(&h);
-    h = __hsub2(*reinterpret_cast<const __half2*>(&p23), off); r.y = *reinterpret_cast<uint32_t*>(&h);
-    h = __hsub2(*reinterpret_cast<const __half2*>(&p45), off); r.z = *reinterpret_cast<uint32_t*>(&h);
-    h = __hsub2(*reinterpret_cast<const __half2*>(&p67), off); r.w = *reinterpret_cast<uint32_t*>(&h);
+    h = __hsub2(*reinterpret_cast<const __half2*>(&e04), off); r.x = *reinterpret_cast<uint32_t*>(&h);
+    h = __hfma2(*reinterpret_cast<const __half2*>(&e15), sixteenth, m72); r.y = *reinterpret_cast<uint32_t*>(&h);
+    h = __hsub2(*reinterpret_cast<const __half2*>(&e26), off); r.z = *reinterpret_cast<uint32_t*>(&h);
+    h = __hfma2(*reinterpret_cast<const __half2*>(&e37), sixteenth, m72); r.w = *reinterpret_cast<uint32_t*>(&h);
     return r;
 }
 
@@ -146,7 +185,8 @@ __device__ __forceinline__ void fold2(float2& acc, uint32_t v0, uint32_t v1, flo
 }
 
 // Q8_0 of 32 values held by one thread, same arithmetic as q8_0_lane; the codes
-// are returned as fp16 pairs (exact) for the down GEMM.
+// are returned as fp16 pairs (exact) for the down GEMM, each group of 8 in the
+// order 0 4 1 5 2 6 3 7.
 __device__ __forceinline__ float q8_0_thread_f16(const float (&v)[32], uint32_t (&codes)[16]) {
     float amax = 0.0f;
 #pragma unroll
@@ -154,11 +194,12 @@ __device__ __forceinline__ float q8_0_thread_f16(const float (&v)[32], uint32_t 
     const float d = __fdiv_rn(amax, 127.0f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
+        const int e = 8 * (j >> 2) + (j & 3);  // group element pair (e, e + 4)
         float q[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             q[i] = 0.0f;
-            if (d != 0.0f) q[i] = fminf(fmaxf(roundf(__fdiv_rn(v[2 * j + i], d)), -127.0f), 127.0f);
+            if (d != 0.0f) q[i] = fminf(fmaxf(roundf(__fdiv_rn(v[e + 4 * i], d)), -127.0f), 127.0f);
         }
         const __half2 h = __floats2half2_rn(q[0], q[1]);
         codes[j] = *reinterpret_cast<const uint32_t*>(&h);
@@ -168,7 +209,7 @@ __device__ __forceinline__ float q8_0_thread_f16(const float (&v)[32], uint32_t 
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreadsG, 1)
-    k_moe_gemm(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tm_a,
+    k_moe_gemm(const __grid_constant__ GemmParams p, const __grid_constant__ RowMaps tm_a,
                const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                const __grid_constant__ CUtensorMap tm_b0s, const __grid_constant__ CUtensorMap tm_b1s) {
     extern __shared__ __align__(1024) uint8_t gsm_raw[];
@@ -198,8 +239,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     const int n_items = U + (p.has_shared ? 1 : 0);
     if (tid == 0) {
         for (int i = 0; i < kStagesG; ++i) {
-            // up/gate: the producer lanes' cp.async arrivals plus the weights' TMA bytes
-            mbar_init(&s.full[i], MODE == kGemmUpGate ? 1 + 32 : 1);
+            mbar_init(&s.full[i], 1);
             mbar_init(&s.bready[i], kXformWarps);
             mbar_init(&s.empty[i], 1);
         }
@@ -237,161 +277,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     const int n_tiles = s.item_tile0[n_items];
     const uint32_t tmem = *s.tmem_base;
 
-    if (warp == kWarpProducer) {
-        // ------------------------------------------------------------ producer
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        long issued = 0;
-        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            int item, nt, mt;
-            tile_of(s, n_items, n_tiles_n, t, item, nt, mt);
-            const Item it = item_of(p, U, item);
-            const int r0 = it.row0 + mt * kBM;
-            const int rows = min(kBM, it.rows - mt * kBM);
-            const __half* arow[4];  // up/gate: this lane's gathered activation rows
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = lane + 32 * j;
-                arow[j] = nullptr;
-                if (MODE == kGemmUpGate && r < rows) {
-                    const int tk = it.shared ? (r0 - p.P + r) : p.pair_tok[r0 + r];
-                    arow[j] = static_cast<const __half*>(p.a_codes) + static_cast<size_t>(tk) * kdim;
-                }
-            }
-            const CUtensorMap* b0 = it.shared ? &tm_b0s : &tm_b0;
-            const CUtensorMap* b1 = it.shared ? &tm_b1s : &tm_b1;
-            const int wr = (it.shared ? 0 : it.e * nout) + nt * cols_per_tile;
-            for (int ks = 0; ks < ksteps; ++ks) {
-                if (!gwait(&s.empty[stage], phase ^ 1u, p.status)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* st = s.stage + stage * kStageBytesG;
-                uint8_t* a = st;
-                uint8_t* packed = st + 2 * kTileBytes;
-                const uint32_t a_bytes = MODE == kGemmUpGate ? 0u : static_cast<uint32_t>(kTileBytes);
-                if (lane == 0) mbar_arrive_expect_tx(&s.full[stage], a_bytes + kPackedBytes);
-                __syncwarp();
-                if (MODE == kGemmUpGate) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int r = lane + 32 * j;
-                        if (arow[j]) {
-                            const __half* src = arow[j] + ks * kBK;
-#pragma unroll
-                            for (int c = 0; c < kBK / 8; ++c) cp_async_16(a + sw128_off(r, c), src + 8 * c);
-                        }
-                    }
-                    cp_async_arrive_noinc(&s.full[stage]);
-                    if (lane == 0) {  // gate rows then up rows, 64 each
-                        tma_load_2d(packed, b0, ks * (kBK / 2), wr, &s.full[stage]);
-                        tma_load_2d(packed + kPackedBytes / 2, b1, ks * (kBK / 2), wr, &s.full[stage]);
-                    }
-                } else if (lane == 0) {
-                    tma_load_2d(a, &tm_a, ks * kBK, r0, &s.full[stage]);
-                    tma_load_2d(packed, b0, ks * (kBK / 2), wr, &s.full[stage]);
-                }
-                ++issued;
-                if (++stage == kStagesG) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-        // drain: every copy issued into this CTA's shared memory has landed
-        if (lane == 0) {
-            for (int st = 0; st < kStagesG; ++st) {
-                const long uses = issued / kStagesG + (st < issued % kStagesG ? 1 : 0);
-                if (uses > 0) mbar_wait(&s.full[st], static_cast<uint32_t>((uses - 1) & 1), kGemmWait);
-            }
-        }
-        __syncwarp();
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            int stage = 0, slot = 0;
-            uint32_t phase = 0, rphase = 0;
-            bool ok = true;
-            const uint32_t idesc = umma_idesc_f16(kBM, kBN);
-            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-                for (int ks = 0; ks < ksteps && ok; ++ks) {
-                    if (!gwait(&s.full[stage], phase, p.status) || !gwait(&s.bready[stage], phase, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint8_t* st = s.stage + stage * kStageBytesG;
-                    const uint8_t* a = st;
-                    const uint8_t* b = st + kTileBytes;
-#pragma unroll
-                    for (int blk = 0; blk < kBK / 32; ++blk) {  // one 32-block per ring slot
-                        if (!gwait(&s.rempty[slot], rphase ^ 1u, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after_sync();
-                        const uint32_t d = tmem + slot * kBN;
-                        umma_f16(d, umma_desc_sw128(a, 64 * blk), umma_desc_sw128(b, 64 * blk), idesc, false);
-                        umma_f16(d, umma_desc_sw128(a, 64 * blk + 32), umma_desc_sw128(b, 64 * blk + 32), idesc,
-                                 true);
-                        umma_commit(&s.rfull[slot]);
-                        if (++slot == kRing) {
-                            slot = 0;
-                            rphase ^= 1u;
-                        }
-                    }
-                    umma_commit(&s.empty[stage]);  // frees the stage once these MMAs are done
-                    if (++stage == kStagesG) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            // every MMA issued by this thread has completed before TMEM is freed
-            umma_commit(s.mma_done);
-            mbar_wait(s.mma_done, 0, kGemmWait);
-        }
-        __syncwarp();
-    } else if (warp < kWarpEpi0) {
-        // ------------------------------------------------------------ dequantise weights
-        const int xt = tid - kWarpXform0 * 32;  // 0 .. 32 kXformWarps - 1
-        int stage = 0;
-        uint32_t phase = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-            for (int ks = 0; ks < ksteps; ++ks) {
-                if (!gwait(&s.full[stage], phase, p.status)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* st = s.stage + stage * kStageBytesG;
-                uint8_t* b = st + kTileBytes;
-                const uint8_t* packed = st + 2 * kTileBytes;
-                // B row br <- packed row: up/gate interleaves [gate 32 | up 32 | gate 32 | up 32]
-                // so that each epilogue warp's 64 columns hold gate and up of the same 32 h
-                for (int task = xt; task < kBN * 2; task += 32 * kXformWarps) {
-                    const int br = task >> 1, hv = task & 1;  // hv: chunks 0-3 or 4-7 of the row
-                    int src_row = br;
-                    if (MODE == kGemmUpGate) src_row = ((br >> 5) & 1) * 64 + (br & 31) + ((br >> 6) << 5);
-                    const uint4 w = reinterpret_cast<const uint4*>(packed + src_row * (kBK / 2))[hv];
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        *reinterpret_cast<uint4*>(b + sw128_off(br, 4 * hv + c)) = int4x8_to_f16(ws[c]);
-                }
-                // orders the dequantised weights, and the activation rows copied by
-                // cp.async (complete once `full` was observed), before the MMAs
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.bready[stage]);
-                if (++stage == kStagesG) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    } else {
+    if (warp >= kWarpEpi0) {
+        regs_raise<kRegsHigh>();
         // ------------------------------------------------------------ epilogue
         const int eh = warp - kWarpEpi0;            // 0..7
         const int q = warp & 3;                     // TMEM lane quarter of this warp
@@ -413,27 +300,29 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 slot_k = it.shared ? 0 : p.pair_slot[pr];
                 arow = MODE == kGemmUpGate ? tok : pr;
             }
-            const float* drow = p.a_scales + static_cast<size_t>(arow) * nblk;
+            // the two block scales of each k step (nblk is even), prefetched kPre steps ahead
+            const float2* d2 = reinterpret_cast<const float2*>(p.a_scales + static_cast<size_t>(arow) * nblk);
             float2 acc[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
-            float dnext = __ldg(drow);
-            for (int b = 0; b < nblk; ++b) {
-                const float db = dnext;
-                if (b + 1 < nblk) dnext = __ldg(drow + b + 1);
-                if (!gwait(&s.rfull[slot], rphase, p.status)) {
-                    ok = false;
-                    break;
-                }
+            constexpr int kPre = 4;
+            float2 dq[kPre];
+#pragma unroll
+            for (int j = 0; j < kPre; ++j) dq[j] = j < ksteps ? __ldg(d2 + j) : make_float2(0.0f, 0.0f);
+            // Software pipeline over the tile's blocks: the TMEM loads of block
+            // b + 1 are in flight while block b is folded, and a ring slot is
+            // released as soon as its values are in registers.
+            const uint32_t lane_off = half * 64 + (static_cast<uint32_t>(q * 32) << 16);
+            uint32_t va[64], vb[64];
+            auto load_block = [&](uint32_t (&v)[64]) -> bool {
+                if (!gwait(&s.rfull[slot], rphase, p.status)) return false;
                 tc_fence_after_sync();
-                const uint32_t ta = tmem + slot * kBN + half * 64 + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(ta + 32 * c, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) fold2(acc[16 * c + i], v[2 * i], v[2 * i + 1], db);
-                }
+                const uint32_t ta = tmem + slot * kBN + lane_off;
+                tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                return true;
+            };
+            auto release_block = [&]() {  // after tmem_wait_ld: the slot's values are in registers
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s.rempty[slot]);
@@ -441,7 +330,42 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                     slot = 0;
                     rphase ^= 1u;
                 }
+            };
+            auto fold_block = [&](const uint32_t (&v)[64], float db) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) fold2(acc[i], v[2 * i], v[2 * i + 1], db);
+            };
+            ok = load_block(va);
+            tmem_wait_ld();
+            if (ok) release_block();
+            for (int ks0 = 0; ks0 < ksteps && ok; ks0 += kPre) {
+#pragma unroll
+                for (int j = 0; j < kPre; ++j) {
+                    const int ks = ks0 + j;
+                    if (ks >= ksteps || !ok) continue;
+                    const float2 dk = dq[j];
+                    if (ks + kPre < ksteps) dq[j] = __ldg(d2 + ks + kPre);
+                    // block 2 ks is in va; load block 2 ks + 1 into vb
+                    if (!load_block(vb)) {
+                        ok = false;
+                        continue;
+                    }
+                    fold_block(va, dk.x);
+                    tmem_wait_ld();
+                    release_block();
+                    const bool more = ks + 1 < ksteps;
+                    if (more && !load_block(va)) {
+                        ok = false;
+                        continue;
+                    }
+                    fold_block(vb, dk.y);
+                    if (more) {
+                        tmem_wait_ld();
+                        release_block();
+                    }
+                }
             }
+            tmem_wait_ld();
             if (!ok || !valid) continue;
             const int c0 = nt * cols_per_tile + half * (MODE == kGemmUpGate ? 32 : 64);
             if (c0 >= nout) continue;
@@ -481,6 +405,142 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 }
             }
         }
+    } else {
+        regs_lower<kRegsLow>();
+        if (warp == kWarpProducer) {
+            // ------------------------------------------------------------ producer
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            long issued = 0;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                int item, nt, mt;
+                tile_of(s, n_items, n_tiles_n, t, item, nt, mt);
+                const Item it = item_of(p, U, item);
+                const int r0 = it.row0 + mt * kBM;
+                const int rcls = (min(kBM, it.rows - mt * kBM) + 15) / 16 - 1;  // tile height class
+                const uint32_t a_bytes = static_cast<uint32_t>(rcls + 1) * 16u * kBK * 2u;
+                const CUtensorMap* b0 = it.shared ? &tm_b0s : &tm_b0;
+                const CUtensorMap* b1 = it.shared ? &tm_b1s : &tm_b1;
+                const int wr = (it.shared ? 0 : it.e * nout) + nt * cols_per_tile;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (!gwait(&s.empty[stage], phase ^ 1u, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = s.stage + stage * kStageBytesG;
+                    uint8_t* a = st;
+                    uint8_t* packed = st + 2 * kTileBytes;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&s.full[stage], a_bytes + kPackedBytes);
+                        tma_load_2d(a, &tm_a.m[rcls], ks * kBK, r0, &s.full[stage]);
+                        if (MODE == kGemmUpGate) {  // gate rows then up rows, 64 each
+                            tma_load_2d(packed, b0, ks * (kBK / 2), wr, &s.full[stage]);
+                            tma_load_2d(packed + kPackedBytes / 2, b1, ks * (kBK / 2), wr, &s.full[stage]);
+                        } else {
+                            tma_load_2d(packed, b0, ks * (kBK / 2), wr, &s.full[stage]);
+                        }
+                    }
+                    __syncwarp();
+                    ++issued;
+                    if (++stage == kStagesG) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // drain: every copy issued into this CTA's shared memory has landed
+            if (lane == 0) {
+                for (int st = 0; st < kStagesG; ++st) {
+                    const long uses = issued / kStagesG + (st < issued % kStagesG ? 1 : 0);
+                    if (uses > 0) mbar_wait(&s.full[st], static_cast<uint32_t>((uses - 1) & 1), kGemmWait);
+                }
+            }
+            __syncwarp();
+        } else if (warp == kWarpMma) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                int stage = 0, slot = 0;
+                uint32_t phase = 0, rphase = 0;
+                bool ok = true;
+                const uint32_t idesc = umma_idesc_f16(kBM, kBN);
+                for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                    for (int ks = 0; ks < ksteps && ok; ++ks) {
+                        if (!gwait(&s.full[stage], phase, p.status) || !gwait(&s.bready[stage], phase, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                        const uint8_t* st = s.stage + stage * kStageBytesG;
+                        const uint8_t* a = st;
+                        const uint8_t* b = st + kTileBytes;
+    #pragma unroll
+                        for (int blk = 0; blk < kBK / 32; ++blk) {  // one 32-block per ring slot
+                            if (!gwait(&s.rempty[slot], rphase ^ 1u, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after_sync();
+                            const uint32_t d = tmem + slot * kBN;
+                            umma_f16(d, umma_desc_sw128(a, 64 * blk), umma_desc_sw128(b, 64 * blk), idesc, false);
+                            umma_f16(d, umma_desc_sw128(a, 64 * blk + 32), umma_desc_sw128(b, 64 * blk + 32), idesc,
+                                     true);
+                            umma_commit(&s.rfull[slot]);
+                            if (++slot == kRing) {
+                                slot = 0;
+                                rphase ^= 1u;
+                            }
+                        }
+                        umma_commit(&s.empty[stage]);  // frees the stage once these MMAs are done
+                        if (++stage == kStagesG) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+                // every MMA issued by this thread has completed before TMEM is freed
+                umma_commit(s.mma_done);
+                mbar_wait(s.mma_done, 0, kGemmWait);
+            }
+            __syncwarp();
+        } else if (warp < kWarpXform0 + kXformWarps) {
+            // ------------------------------------------------------------ dequantise weights
+            const int xt = tid - kWarpXform0 * 32;  // 0 .. 32 kXformWarps - 1
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    if (!gwait(&s.full[stage], phase, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* st = s.stage + stage * kStageBytesG;
+                    uint8_t* b = st + kTileBytes;
+                    const uint8_t* packed = st + 2 * kTileBytes;
+                    // B row br <- packed row: up/gate interleaves [gate 32 | up 32 | gate 32 | up 32]
+                    // so that each epilogue warp's 64 columns hold gate and up of the same 32 h
+                    for (int task = xt; task < kBN * 2; task += 32 * kXformWarps) {
+                        const int br = task >> 1, hv = task & 1;  // hv: chunks 0-3 or 4-7 of the row
+                        int src_row = br;
+                        if (MODE == kGemmUpGate) src_row = ((br >> 5) & 1) * 64 + (br & 31) + ((br >> 6) << 5);
+                        const uint4 w = reinterpret_cast<const uint4*>(packed + src_row * (kBK / 2))[hv];
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    #pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4*>(b + sw128_off(br, 4 * hv + c)) = int4x8_to_f16(ws[c]);
+                    }
+                    // orders the dequantised weights before the MMAs (async proxy)
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.bready[stage]);
+                    if (++stage == kStagesG) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
     }
     tc_fence_before_sync();
     __syncthreads();
@@ -490,18 +550,24 @@ __global__ void __launch_bounds__(kThreadsG, 1)
     }
 }
 
-// Activation codes as fp16 (exact): one thread per 8 codes.
-__global__ void k_codes_f16(const int8_t* __restrict__ q, size_t n8, __half* __restrict__ out) {
+// The up/gate GEMM's activation rows: row r < P is the Q8_0 codes of token
+// pair_tok[r] (union order), row P + t those of token t (shared expert); codes
+// as fp16 (exact), each group of 8 in the order 0 4 1 5 2 6 3 7.  One thread
+// per group of 8.
+__global__ void k_gather_codes(const int8_t* __restrict__ q, int H, int P, size_t rows,
+                               const int32_t* __restrict__ pair_tok, __half* __restrict__ out) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= n8) return;
-    const uint2 raw = reinterpret_cast<const uint2*>(q)[i];
-    const uint32_t w[2] = {raw.x, raw.y};
+    const int g = H / 8;
+    if (i >= rows * g) return;
+    const size_t r = i / g;
+    const int c = static_cast<int>(i - r * g);
+    const int tok = r < static_cast<size_t>(P) ? __ldg(pair_tok + r) : static_cast<int>(r - P);
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(q + static_cast<size_t>(tok) * H) + c);
+    auto code = [&](int e) { return static_cast<float>(static_cast<int8_t>(((e < 4 ? raw.x : raw.y) >> (8 * (e & 3))) & 0xFF)); };
     uint32_t o[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int a = static_cast<int8_t>((w[j >> 1] >> (16 * (j & 1))) & 0xFF);
-        const int b = static_cast<int8_t>((w[j >> 1] >> (16 * (j & 1) + 8)) & 0xFF);
-        const __half2 h = __floats2half2_rn(static_cast<float>(a), static_cast<float>(b));
+        const __half2 h = __floats2half2_rn(code(j), code(j + 4));
         o[j] = *reinterpret_cast<const uint32_t*>(&h);
     }
     reinterpret_cast<uint4*>(out)[i] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -551,16 +617,19 @@ bool tc_gemm_supported(const moe_experts& r, const moe_experts* s, int E) {
     return true;
 }
 
-cudaError_t launch_codes_f16(const int8_t* q, size_t n, __half* out, cudaStream_t st) {
-    const size_t n8 = n / 8;
+cudaError_t launch_gather_codes(const int8_t* q, int H, int P, int rows, const int32_t* pair_tok, __half* out,
+                                cudaStream_t st) {
+    const size_t n8 = static_cast<size_t>(rows) * (H / 8);
     if (n8 == 0) return cudaSuccess;
     const int threads = 256;
-    k_codes_f16<<<static_cast<unsigned>((n8 + threads - 1) / threads), threads, 0, st>>>(q, n8, out);
+    k_gather_codes<<<static_cast<unsigned>((n8 + threads - 1) / threads), threads, 0, st>>>(q, H, P, rows, pair_tok,
+                                                                                            out);
     return counted(cudaGetLastError());
 }
 
 cudaError_t launch_moe_gemm(int mode, const GemmParams& p, const GemmOperands& o, cudaStream_t st) {
-    CUtensorMap a, b0, b1, b0s, b1s;
+    RowMaps a;
+    CUtensorMap b0, b1, b0s, b1s;
     const int K = mode == kGemmUpGate ? p.H : p.I;  // contraction
     const int nout = mode == kGemmUpGate ? p.I : p.H;
     const uint32_t brows = mode == kGemmUpGate ? kBN / 2 : kBN;
@@ -579,13 +648,13 @@ cudaError_t launch_moe_gemm(int mode, const GemmParams& p, const GemmOperands& o
                           CU_TENSOR_MAP_SWIZZLE_NONE);
         else
             b1s = b1;
-        a = b0;  // up/gate gathers its activation rows with cp.async: no map
     } else {
         b1 = b0;
         b1s = b0s;
-        ok = ok && make_map(&a, p.a_codes, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K,
-                            static_cast<uint64_t>(p.P + p.T), kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
     }
+    for (int c = 0; c < kRowClasses && ok; ++c)
+        ok = make_map(&a.m[c], p.a_codes, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, static_cast<uint64_t>(p.P + p.T), kBK,
+                      16 * (c + 1), CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     static int sms[64] = {0};
     int dev = 0;
@@ -601,6 +670,11 @@ cudaError_t launch_moe_gemm(int mode, const GemmParams& p, const GemmOperands& o
                                            : reinterpret_cast<const void*>(k_moe_gemm<kGemmDown>);
     e = ensure_smem(kern, smem);
     if (e != cudaSuccess) return e;
+    // the in-kernel register split assumes this launch size exactly
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     if (mode == kGemmUpGate)
         k_moe_gemm<kGemmUpGate><<<grid, kThreadsG, smem, st>>>(p, a, b0, b1, b0s, b1s);
     else
