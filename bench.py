@@ -61,7 +61,7 @@ def tensor_peak():
         return 1590.0, "fallback"
 
 
-KERNEL_SOURCES = ("decode_fused.cu", "common.cuh", "kernels.cuh", "quant.cuh", "sm100_async.cuh")
+KERNEL_SOURCES = ("decode_fused.cu", "common.cuh", "quant.cuh", "sm100_async.cuh")
 
 
 def profiled_traffic():
