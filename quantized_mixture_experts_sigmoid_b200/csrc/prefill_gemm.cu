@@ -13,9 +13,12 @@
 // both operands are the integer codes written as fp16 (exact: |q| <= 127 and
 // the int4 weight codes), one 32-element block per pair of K = 16 MMAs; the
 // fp32 accumulator of a block holds an integer below 2^15 (exact).  Each
-// block's result lands in its own slot of a 4-slot TMEM ring; the epilogue
-// warps fold it into per-thread fp32 accumulators in block order (packed
-// f32x2 fused multiply-add).  Up/gate then applies SwiGLU and Q8_0 to h (the
+// block's result lands in its own TMEM slot; the two blocks of a 64-K stage
+// form a slot pair, and the ring holds two pairs.  One tcgen05.commit per
+// stage (on the stage's `empty` barrier) tells both the producer that the
+// stage's shared memory is free and the epilogue that the pair's results are
+// in TMEM; the epilogue warps fold them into per-thread fp32 accumulators in
+// block order (packed f32x2 fused multiply-add).  Up/gate then applies SwiGLU and Q8_0 to h (the
 // codes written as fp16 for the down GEMM); down writes the fp32 output per
 // (token, slot).  The result is the same, bit for bit, as the reference
 // arithmetic.
@@ -53,6 +56,7 @@ constexpr int kBN = 128;            // MMA columns per tile
 constexpr int kBK = 64;             // K per stage (one 128-byte swizzle atom of fp16) = 2 blocks
 constexpr int kStagesG = 6;
 constexpr int kRing = 4;            // TMEM slots of block results (kRing x kBN columns)
+constexpr int kPairs = kRing / 2;   // slot pairs: the two blocks of one stage
 constexpr int kThreadsG = 512;
 constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpXform0 = 2, kXformWarps = 4, kWarpEpi0 = 8, kEpiWarps = 8;
 // Register split: the CTA is launched with kLaunchRegs per thread (checked on
@@ -82,8 +86,7 @@ struct GemmSmem {
     uint64_t* full;       // [kStagesG] activation and weight bytes landed
     uint64_t* bready;     // [kStagesG] weights dequantised
     uint64_t* empty;      // [kStagesG] MMAs done with the stage
-    uint64_t* rfull;      // [kRing] block result ready in TMEM
-    uint64_t* rempty;     // [kRing] block result folded by every epilogue warp
+    uint64_t* rempty;     // [kPairs] slot pair read out by every epilogue warp
     uint64_t* mma_done;   // every MMA of this CTA has completed
     uint32_t* tmem_base;
     int* item_tile0;      // [kMaxItems + 1] first tile of each expert item
@@ -222,9 +225,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         s.full = bars;
         s.bready = bars + kStagesG;
         s.empty = bars + 2 * kStagesG;
-        s.rfull = bars + 3 * kStagesG;
-        s.rempty = s.rfull + kRing;
-        s.mma_done = s.rempty + kRing;
+        s.rempty = bars + 3 * kStagesG;
+        s.mma_done = s.rempty + kPairs;
         s.tmem_base = reinterpret_cast<uint32_t*>(s.mma_done + 1);
         s.item_tile0 = reinterpret_cast<int*>(s.tmem_base + 4);
     }
@@ -243,10 +245,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             mbar_init(&s.bready[i], kXformWarps);
             mbar_init(&s.empty[i], 1);
         }
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(&s.rfull[i], 1);
-            mbar_init(&s.rempty[i], kEpiWarps);
-        }
+        for (int i = 0; i < kPairs; ++i) mbar_init(&s.rempty[i], kEpiWarps);
         mbar_init(s.mma_done, 1);
         fence_mbar_init();
     }
@@ -284,8 +283,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         const int q = warp & 3;                     // TMEM lane quarter of this warp
         const int half = eh >> 2;                   // columns 64 half .. 64 half + 63 of each slot
         const int r = q * 32 + lane;                // tile row (token / pair) of this thread
-        int slot = 0;
-        uint32_t rphase = 0;
+        int stage = 0, pair = 0;                    // the MMA issuer's stage / slot-pair sequence
+        uint32_t phase = 0, rphase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             int item, nt, mt;
@@ -309,35 +308,9 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             float2 dq[kPre];
 #pragma unroll
             for (int j = 0; j < kPre; ++j) dq[j] = j < ksteps ? __ldg(d2 + j) : make_float2(0.0f, 0.0f);
-            // Software pipeline over the tile's blocks: the TMEM loads of block
-            // b + 1 are in flight while block b is folded, and a ring slot is
-            // released as soon as its values are in registers.
+            // Per stage: wait for the MMAs' commit on the stage's `empty` barrier,
+            // load the pair's two block results, release the pair, fold both.
             const uint32_t lane_off = half * 64 + (static_cast<uint32_t>(q * 32) << 16);
-            uint32_t va[64], vb[64];
-            auto load_block = [&](uint32_t (&v)[64]) -> bool {
-                if (!gwait(&s.rfull[slot], rphase, p.status)) return false;
-                tc_fence_after_sync();
-                const uint32_t ta = tmem + slot * kBN + lane_off;
-                tmem_ld32_async(ta, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                tmem_ld32_async(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                return true;
-            };
-            auto release_block = [&]() {  // after tmem_wait_ld: the slot's values are in registers
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.rempty[slot]);
-                if (++slot == kRing) {
-                    slot = 0;
-                    rphase ^= 1u;
-                }
-            };
-            auto fold_block = [&](const uint32_t (&v)[64], float db) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) fold2(acc[i], v[2 * i], v[2 * i + 1], db);
-            };
-            ok = load_block(va);
-            tmem_wait_ld();
-            if (ok) release_block();
             for (int ks0 = 0; ks0 < ksteps && ok; ks0 += kPre) {
 #pragma unroll
                 for (int j = 0; j < kPre; ++j) {
@@ -345,27 +318,39 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                     if (ks >= ksteps || !ok) continue;
                     const float2 dk = dq[j];
                     if (ks + kPre < ksteps) dq[j] = __ldg(d2 + ks + kPre);
-                    // block 2 ks is in va; load block 2 ks + 1 into vb
-                    if (!load_block(vb)) {
+                    if (!gwait(&s.empty[stage], phase, p.status)) {
                         ok = false;
                         continue;
                     }
-                    fold_block(va, dk.x);
+                    tc_fence_after_sync();
+                    const uint32_t ta = tmem + pair * 2 * kBN + lane_off;
+                    uint32_t va[32], vb[32], vc[32], vd[32];
+                    tmem_ld32_async(ta, va);
+                    tmem_ld32_async(ta + 32, vb);
+                    tmem_ld32_async(ta + kBN, vc);
+                    tmem_ld32_async(ta + kBN + 32, vd);
                     tmem_wait_ld();
-                    release_block();
-                    const bool more = ks + 1 < ksteps;
-                    if (more && !load_block(va)) {
-                        ok = false;
-                        continue;
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.rempty[pair]);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) fold2(acc[i], va[2 * i], va[2 * i + 1], dk.x);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) fold2(acc[16 + i], vb[2 * i], vb[2 * i + 1], dk.x);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) fold2(acc[i], vc[2 * i], vc[2 * i + 1], dk.y);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) fold2(acc[16 + i], vd[2 * i], vd[2 * i + 1], dk.y);
+                    if (++stage == kStagesG) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
-                    fold_block(vb, dk.y);
-                    if (more) {
-                        tmem_wait_ld();
-                        release_block();
+                    if (++pair == kPairs) {
+                        pair = 0;
+                        rphase ^= 1u;
                     }
                 }
             }
-            tmem_wait_ld();
             if (!ok || !valid) continue;
             const int c0 = nt * cols_per_tile + half * (MODE == kGemmUpGate ? 32 : 64);
             if (c0 >= nout) continue;
@@ -460,7 +445,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
         } else if (warp == kWarpMma) {
             // ------------------------------------------------------------ MMA issuer
             if (lane == 0) {
-                int stage = 0, slot = 0;
+                int stage = 0, pair = 0;
                 uint32_t phase = 0, rphase = 0;
                 bool ok = true;
                 const uint32_t idesc = umma_idesc_f16(kBM, kBN);
@@ -470,28 +455,28 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                             ok = false;
                             break;
                         }
+                        if (!gwait(&s.rempty[pair], rphase ^ 1u, p.status)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after_sync();
                         const uint8_t* st = s.stage + stage * kStageBytesG;
                         const uint8_t* a = st;
                         const uint8_t* b = st + kTileBytes;
-    #pragma unroll
-                        for (int blk = 0; blk < kBK / 32; ++blk) {  // one 32-block per ring slot
-                            if (!gwait(&s.rempty[slot], rphase ^ 1u, p.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after_sync();
-                            const uint32_t d = tmem + slot * kBN;
+#pragma unroll
+                        for (int blk = 0; blk < kBK / 32; ++blk) {  // one 32-block per slot of the pair
+                            const uint32_t d = tmem + (2 * pair + blk) * kBN;
                             umma_f16(d, umma_desc_sw128(a, 64 * blk), umma_desc_sw128(b, 64 * blk), idesc, false);
                             umma_f16(d, umma_desc_sw128(a, 64 * blk + 32), umma_desc_sw128(b, 64 * blk + 32), idesc,
                                      true);
-                            umma_commit(&s.rfull[slot]);
-                            if (++slot == kRing) {
-                                slot = 0;
-                                rphase ^= 1u;
-                            }
                         }
-                        umma_commit(&s.empty[stage]);  // frees the stage once these MMAs are done
+                        // one commit: the stage's shared memory is free (producer) and the
+                        // pair's results are in TMEM (epilogue)
+                        umma_commit(&s.empty[stage]);
+                        if (++pair == kPairs) {
+                            pair = 0;
+                            rphase ^= 1u;
+                        }
                         if (++stage == kStagesG) {
                             stage = 0;
                             phase ^= 1u;
@@ -526,7 +511,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                         if (MODE == kGemmUpGate) src_row = ((br >> 5) & 1) * 64 + (br & 31) + ((br >> 6) << 5);
                         const uint4 w = reinterpret_cast<const uint4*>(packed + src_row * (kBK / 2))[hv];
                         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    #pragma unroll
+#pragma unroll
                         for (int c = 0; c < 4; ++c)
                             *reinterpret_cast<uint4*>(b + sw128_off(br, 4 * hv + c)) = int4x8_to_f16(ws[c]);
                     }
