@@ -449,6 +449,10 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 uint32_t phase = 0, rphase = 0;
                 bool ok = true;
                 const uint32_t idesc = umma_idesc_f16(kBM, kBN);
+                // descriptors of stage 0; a stage or K offset adds (bytes >> 4) to the
+                // start-address field (all addresses stay below 256 KiB)
+                const uint64_t adesc0 = umma_desc_sw128(s.stage, 0);
+                const uint64_t bdesc0 = umma_desc_sw128(s.stage + kTileBytes, 0);
                 for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                     for (int ks = 0; ks < ksteps && ok; ++ks) {
                         if (!gwait(&s.full[stage], phase, p.status) || !gwait(&s.bready[stage], phase, p.status)) {
@@ -460,16 +464,14 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                             break;
                         }
                         tc_fence_after_sync();
-                        const uint8_t* st = s.stage + stage * kStageBytesG;
-                        const uint8_t* a = st;
-                        const uint8_t* b = st + kTileBytes;
-#pragma unroll
-                        for (int blk = 0; blk < kBK / 32; ++blk) {  // one 32-block per slot of the pair
-                            const uint32_t d = tmem + (2 * pair + blk) * kBN;
-                            umma_f16(d, umma_desc_sw128(a, 64 * blk), umma_desc_sw128(b, 64 * blk), idesc, false);
-                            umma_f16(d, umma_desc_sw128(a, 64 * blk + 32), umma_desc_sw128(b, 64 * blk + 32), idesc,
-                                     true);
-                        }
+                        const uint64_t soff = static_cast<uint64_t>((stage * kStageBytesG) >> 4);
+                        const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
+                        const uint32_t d = tmem + pair * 2 * kBN;
+                        // block 0 (K 0..31 of the stage) into the pair's first slot, block 1 into the second
+                        umma_f16(d, ad, bd, idesc, false);
+                        umma_f16(d, ad + 2, bd + 2, idesc, true);
+                        umma_f16(d + kBN, ad + 4, bd + 4, idesc, false);
+                        umma_f16(d + kBN, ad + 6, bd + 6, idesc, true);
                         // one commit: the stage's shared memory is free (producer) and the
                         // pair's results are in TMEM (epilogue)
                         umma_commit(&s.empty[stage]);
