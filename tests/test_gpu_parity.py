@@ -37,17 +37,19 @@ SHAPES = {
                                           topk_group=2, top_k=6, qtype=2),
     "fused_ragged_int8": synth.LayerShape("fused_ragged_int8", T=4, H=544, I=288, E=96, n_group=3,
                                           topk_group=2, top_k=5, qtype=8),
-    # many tokens per expert on the tensor cores: several 128-row tiles per
-    # expert, ragged N and K tails (I = 192, H = 320), shared expert included
+    # batches on the tensor cores: ragged N and K tails (I = 192, H = 320), partial 128-row
+    # tiles of every height class, shared expert included; tc_multi gives every expert
+    # about 160 pairs (two row tiles, the second partial) and the shared expert five
     "tc_small": synth.LayerShape("tc_small", T=40, H=256, I=128, E=16, n_group=4, topk_group=2, top_k=4),
     "tc_ragged": synth.LayerShape("tc_ragged", T=300, H=320, I=192, E=32, n_group=4, topk_group=2, top_k=6),
+    "tc_multi": synth.LayerShape("tc_multi", T=640, H=320, I=192, E=16, n_group=4, topk_group=2, top_k=4),
     "decode": synth.CONFIGS["decode"],
     "verify": synth.CONFIGS["verify"],
     "verify_int8": synth.CONFIGS["verify_int8"],
     "decode_int2": synth.CONFIGS["decode"].with_(qtype=2, name="decode_int2"),
 }
 SMALL = ["tiny", "ragged", "crowded", "crowded_int8", "crowded_int2", "fused_ragged",
-         "fused_ragged_int2", "fused_ragged_int8", "tc_small", "tc_ragged"]
+         "fused_ragged_int2", "fused_ragged_int8", "tc_small", "tc_ragged", "tc_multi"]
 FULL = ["decode", "verify", "verify_int8", "decode_int2"]
 
 _cache = {}
@@ -270,6 +272,14 @@ def test_layer_forward_without_shared_and_empty_batch():
                           dev["shared"], out, ws)
 
 
+def test_tensor_core_path_without_shared_expert():
+    # no shared rows: the gathered activation buffer and the tile list stop at the pairs
+    sh, dev = layer("tc_multi")
+    assert moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], None) == moe.PATH_TENSOR_CORE
+    x, W, b = layer_inputs(sh)
+    check_layer(sh, dev, x, W, b, shared=False)
+
+
 def test_union_path_equals_per_token_path_on_gpu():
     # draft and verify must compute the same function (molayo1419.me, section
     # "정직하게 구현된 투기적 디코딩"): a token's output does not depend on which
@@ -294,7 +304,7 @@ def test_union_path_equals_sub_batches_on_tensor_cores():
 
 
 FUSED = ["fused_ragged", "fused_ragged_int2", "fused_ragged_int8", "decode", "verify", "decode_int2"]
-TENSOR_CORE = ["tc_small", "tc_ragged"]
+TENSOR_CORE = ["tc_small", "tc_ragged", "tc_multi"]
 
 
 @pytest.mark.parametrize("name", FUSED + TENSOR_CORE + ["tiny", "ragged", "crowded_int8"])
