@@ -128,8 +128,8 @@ def oracle_sample(sh, seconds: float, first_token: int = 0, max_tokens: int | No
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    _, rank, _ = rank_env()
+    if rank != 0:  # the oracle runs once, on rank 0; the other ranks exit without work
         return
     sh = synth.CONFIGS["decode"]
     # one step = one token's full layer on the CPU oracle; warm-up and timed
@@ -197,6 +197,27 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CUDA arm
+def rank_env():
+    """(world size, rank, local rank) from the torchrun environment; (1, 0, 0) without it."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of every rank's value (a device time): all ranks call it in the same order."""
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_tokens_per_s(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput of `world` replicas, each running `steps` steps, timed by the slowest."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     """The batch-union prefill layer (T = 2048, Zipf-skewed routing) on the tensor-core path:
     whole-layer tokens/s and the two expert GEMMs' share of the dense tensor roofline."""
@@ -270,9 +291,7 @@ def run_cuda(args):
         print(json.dumps(prefill_measurement(args, moe, moe.lib(), device_layer, to_dev_bf16)), flush=True)
         return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -321,10 +340,7 @@ def run_cuda(args):
         wall = time.perf_counter() - wall0
     launches = L.moe_launch_count() - launches0
     dev_ms = ev0.elapsed_time(ev1)
-    t_max = torch.tensor([dev_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    dev_ms = float(t_max.item())
+    dev_ms = max_over_ranks(dev_ms, world, "cuda")
     if moe.moe_workspace_status(ws) != 0:
         raise RuntimeError("device status error during timing")
 
@@ -359,10 +375,7 @@ def run_cuda(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    t_e2e = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t_e2e.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
 
     prefill = prefill_measurement(args, moe, L, device_layer, to_dev_bf16) if args.prefill else None
 
@@ -373,7 +386,7 @@ def run_cuda(args):
         return
 
     ms_step = dev_ms / args.steps
-    tok_s = world * T * args.steps / (dev_ms / 1e3)
+    tok_s = replicas_tokens_per_s(world, T, args.steps, dev_ms)
     U = sh.top_k  # T = 1: every step touches top_k distinct routed experts
     expert_bytes = (U + 1) * sh.expert_bytes()
     layer_bytes = expert_bytes + sh.router_bytes()
@@ -401,7 +414,7 @@ def run_cuda(args):
                      "achieved": dom_gbs, "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": profiled_traffic(),
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
-        "e2e": {"value": world * T * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": replicas_tokens_per_s(world, T, e2e_steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
