@@ -18,10 +18,10 @@
 // stage (on the stage's `empty` barrier) tells both the producer that the
 // stage's shared memory is free and the epilogue that the pair's results are
 // in TMEM; the epilogue warps fold them into per-thread fp32 accumulators in
-// block order (packed f32x2 fused multiply-add).  Up/gate then applies SwiGLU and Q8_0 to h (the
-// codes written as fp16 for the down GEMM); down writes the fp32 output per
-// (token, slot).  The result is the same, bit for bit, as the reference
-// arithmetic.
+// block order (packed f32x2 fused multiply-add).  Up/gate then applies SwiGLU
+// and Q8_0 to h (the codes written as fp16 for the down GEMM); down writes the
+// fp32 output per (token, slot).  The result is the same, bit for bit, as the
+// plain definition above evaluated one row at a time.
 //
 // Operand order along K.  Inside every group of 8 consecutive K positions
 // both operands hold the elements in the order 0 4 1 5 2 6 3 7: the order in
