@@ -263,6 +263,48 @@ def test_qdot_against_fp64_dequantised_dot():
         assert abs(got - ref) <= 1e-5 * scale
 
 
+def _round_f32(q):
+    """The fp32 value nearest the rational q (ties to even), found exactly."""
+    from fractions import Fraction
+    c = np.float32(float(q))
+    best = None
+    for v in (np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))):
+        err = abs(Fraction(float(v)) - q)
+        even = (int(np.float32(v).view(np.uint32)) & 1) == 0
+        key = (err, not even)
+        if best is None or key < best[0]:
+            best = (key, v)
+    return np.float32(best[1])
+
+
+def test_qdot_fold_rounds_once_per_block():
+    # reading of the quantised dot: each block step is the fp32 value nearest
+    # isum_b * d_b + acc (one rounding), blocks ascending, then one rounding of
+    # acc * s.  The steps are computed here with exact rationals; the same data
+    # folded with two roundings per step (multiply, then add) must differ
+    # somewhere, so this pin can tell the two apart.
+    from fractions import Fraction
+    rng = np.random.default_rng(31)
+    n = 1024
+    differs = 0
+    for _ in range(40):
+        codes = rng.integers(-8, 8, n).astype(np.int8)
+        x = rng.standard_normal(n).astype(np.float32)
+        s = np.float32(rng.uniform(0.01, 0.05))
+        qa, da = O.q8_0(x)
+        acc = np.float32(0.0)
+        acc2 = np.float32(0.0)
+        for b in range(n // 32):
+            isum = int(np.dot(codes[32 * b:32 * b + 32].astype(np.int64), qa[32 * b:32 * b + 32].astype(np.int64)))
+            acc = _round_f32(Fraction(isum) * Fraction(float(da[b])) + Fraction(float(acc)))
+            acc2 = np.float32(np.float32(np.float32(isum) * da[b]) + acc2)
+        want = _round_f32(Fraction(float(acc)) * Fraction(float(s)))
+        got = np.float32(O.qdot(codes, s, qa, da))
+        assert got.view(np.uint32) == want.view(np.uint32)
+        differs += int(np.float32(acc2 * s).view(np.uint32) != want.view(np.uint32))
+    assert differs > 0
+
+
 # --------------------------------------------------------------- expert
 def _expert_fp64(sh, layer, eid, x_f32, h_oracle=None):
     """Dense fp64 reformulation: dequantise everything, multiply, SwiGLU, requantise h."""
@@ -280,6 +322,31 @@ def _expert_fp64(sh, layer, eid, x_f32, h_oracle=None):
     qh, dh = O.q8_0(hq_src.astype(np.float32))
     ha = qh.astype(np.float64) * np.repeat(dh.astype(np.float64), 32)
     return Wd @ ha, h, np.abs(Wd) @ np.abs(ha)
+
+
+def test_expert_h_is_fp64_silu_rounded_once_times_u():
+    # reading of SwiGLU: silu(g) = g / (1 + e^-g) evaluated in fp64 and rounded
+    # once to fp32, then times u in fp32.  Here silu is computed to 40 digits
+    # (decimal), rounded to fp64 and then to fp32; g and u come from the pinned
+    # quantised dot.  The expert's h must match for every row.
+    from decimal import Decimal, getcontext
+    getcontext().prec = 40
+    sh = synth.CONFIGS["tiny"]
+    for eid in (0, 5, 11):
+        ex = oracle_experts(sh, [eid])
+        x = synth.hidden_states(sh, tokens=[eid])[0]
+        xf = synth.bf16_to_f32(x).astype(np.float32)
+        _, h = O.expert_token(ex, eid, xf, want_h=True)
+        g_pk, sg = synth.expert_matrix(sh, 0, eid, synth.GATE)
+        u_pk, su = synth.expert_matrix(sh, 0, eid, synth.UP)
+        qa, da = O.q8_0(xf)
+        for r in range(sh.I):  # packed rows [I, row bytes]
+            g = np.float32(O.qdot(O.unpack(g_pk[r], sh.qtype, sh.H), sg[r], qa, da))
+            u = np.float32(O.qdot(O.unpack(u_pk[r], sh.qtype, sh.H), su[r], qa, da))
+            gd = Decimal(float(g))
+            silu = gd / (1 + (-gd).exp())
+            want = np.float32(np.float32(float(silu)) * u)
+            assert np.float32(h[r]).view(np.uint32) == want.view(np.uint32), (eid, r)
 
 
 @pytest.mark.parametrize("qtype", [4, 8, 2])
