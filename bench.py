@@ -218,6 +218,18 @@ def replicas_tokens_per_s(world: int, tokens_per_step: int, steps: int, max_ms: 
     return world * tokens_per_step * steps / (max_ms / 1e3)
 
 
+def layer_roofline_ms(rows_per_expert, expert_bytes: int, flops_per_row: float, hbm_gbs: float,
+                      tensor_tflops: float) -> float:
+    """Roofline time of a batch-union layer: every distinct expert (shared included) is read once
+    and applied to its rows; each takes the longer of its weight stream at the HBM peak and its
+    contractions at the tensor peak (experts with few rows are bandwidth-bound)."""
+    t = 0.0
+    for n in rows_per_expert:
+        if n > 0:
+            t += max(expert_bytes / (hbm_gbs * 1e9), n * flops_per_row / (tensor_tflops * 1e12))
+    return t * 1e3
+
+
 def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     """The batch-union prefill layer (T = 2048, Zipf-skewed routing) on the tensor-core path:
     whole-layer tokens/s and the two expert GEMMs' share of the dense tensor roofline."""
@@ -235,8 +247,10 @@ def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     path = moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"])
     stream = torch.cuda.current_stream()
 
+    idx = torch.empty(sh.T, sh.top_k, dtype=torch.int32, device="cuda")
+
     def fwd():
-        moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+        moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws, idx)
 
     for _ in range(3):
         fwd()
@@ -263,6 +277,9 @@ def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     flops = 2.0 * rows * 3 * sh.H * sh.I  # up, gate and down contractions actually needed
     peak, kind = tensor_peak()
     achieved = flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    counts = np.bincount(idx.cpu().numpy().ravel(), minlength=sh.E).tolist() + [sh.T]  # routed experts + shared
+    hbm, _ = peaks()
+    roof_ms = layer_roofline_ms(counts, sh.expert_bytes(), 2.0 * 3 * sh.H * sh.I, hbm, peak)
     del ws, dev
     torch.cuda.empty_cache()
     return {
@@ -270,6 +287,10 @@ def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
                     "Zipf(1.1) expert popularity",
         "path": {moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core", moe.PATH_GENERAL: "general"}[path],
         "tokens_per_s": sh.T / (layer_ms / 1e3), "ms_per_layer": layer_ms, "layers_timed": reps,
+        "distinct_experts": int(sum(1 for c in counts[:-1] if c > 0)),
+        "layer_roofline": {"ms": roof_ms, "frac": roof_ms / layer_ms,
+                           "definition": "sum over distinct experts (shared included) of max(expert bytes / "
+                                         "measured HBM GB/s, rows x 2*3*H*I FLOP / measured dense TFLOP/s)"},
         "roofline": {"bound": "tensor", "kernel": "k_moe_gemm up/gate + down (both launches)",
                      "achieved": achieved, "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
                      "frac": achieved / peak if achieved else None, "flops_per_layer": flops,

@@ -59,3 +59,13 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+
+
+def test_layer_roofline_takes_the_slower_of_stream_and_contraction():
+    # 18.9 MB at 6550 GB/s = 2.89 us; 64 rows x 75.5 MFLOP at 1670.9 TFLOP/s = 2.89 us
+    eb, fr = 18_915_328, 2.0 * 3 * 6144 * 2048
+    t_stream = eb / 6550.1e9 * 1e3
+    t_row = fr / 1670.9e12 * 1e3
+    assert bench.layer_roofline_ms([1], eb, fr, 6550.1, 1670.9) == pytest.approx(t_stream)
+    assert bench.layer_roofline_ms([2048], eb, fr, 6550.1, 1670.9) == pytest.approx(2048 * t_row)
+    assert bench.layer_roofline_ms([0, 1, 2048], eb, fr, 6550.1, 1670.9) == pytest.approx(t_stream + 2048 * t_row)
