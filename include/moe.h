@@ -198,8 +198,13 @@ size_t moe_expert_ffn_workspace_bytes(const moe_experts* ex, int T, int top_k);
  * dequant-on-use, integer dot against Q8_0 activations; batch-union bullet).
  * For every distinct expert u (uniq[u], pairs offsets[u]..offsets[u+1]):
  *   a = Q8_0(x[t]);  g[r] = s_gate[r] * sum_b d_a[b] * isum_b(q_a, q_gate[r]);
- *   u[r] likewise;   h = g / (1 + e^-g) * u  (fp32);  a' = Q8_0(h);
+ *   u[r] likewise;   h = silu(g) * u;  a' = Q8_0(h);
  *   y[c] = s_down[c] * sum_b d_a'[b] * isum_b(q_a', q_down[c])
+ * where isum_b is the exact integer dot of 32-block b, the sum over b is an
+ * fp32 accumulator starting at 0 that takes one fused multiply-add per block
+ * in ascending b, then one fp32 multiply by the row scale; silu(g) =
+ * g / (1 + e^-g) is evaluated in fp64 and rounded once to fp32, and h is the
+ * fp32 product silu(g) * u.
  * and y_pairs[t][slot][:] = y for each pair (t, slot) of the expert.
  * Pass n_unique = uniq = offsets = pair_tok = pair_slot = NULL to apply expert
  * 0 of `ex` to every token (the shared expert); top_k must then be 1.

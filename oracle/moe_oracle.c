@@ -4,6 +4,13 @@
  *
  * Build: gcc -O2 -std=c99 -ffp-contract=off -fopenmp (no fused multiply-add,
  * so every "a * b + c" below is two IEEE roundings, exactly as written).
+ *
+ * Two compile-time switches build VARIANTS of the oracle, used only to
+ * measure how much the layer output depends on roundings the pages leave
+ * open (oracle/variant_report.py); the default build defines neither:
+ *   ORACLE_SILU_F32    silu(g) = g / (1 + expf(-g)) in fp32 instead of fp64
+ *   ORACLE_FOLD_MULADD the block fold acc = acc + isum * d (two roundings)
+ *                      instead of one fused multiply-add
  * OpenMP only splits independent output rows / logits across threads; the
  * arithmetic of each row is the single-threaded loop as written.
  */
@@ -299,7 +306,11 @@ float oracle_qdot(const int8_t* wcodes, float w_scale, const int8_t* qa, const f
     for (int b = 0; b < n / 32; ++b) {
         int32_t isum = 0;
         for (int i = 32 * b; i < 32 * b + 32; ++i) isum += (int32_t)qa[i] * (int32_t)wcodes[i];
+#ifdef ORACLE_FOLD_MULADD
+        acc = acc + (float)isum * da[b];  /* variant: two roundings per block */
+#else
         acc = fmaf((float)isum, da[b], acc);  /* one rounding per block */
+#endif
     }
     return acc * w_scale;
 }
@@ -345,7 +356,11 @@ int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* 
             const float g = oracle_qdot(codes, ex->s_gate[e][r], qa, da, H);
             oracle_unpack(ex->w_up[e] + (size_t)r * rb_in, q, H, codes);
             const float u = oracle_qdot(codes, ex->s_up[e][r], qa, da, H);
+#ifdef ORACLE_SILU_F32
+            const float silu = g / (1.0f + expf(-g));  /* variant: fp32 throughout */
+#else
             const float silu = (float)((double)g / (1.0 + exp(-(double)g)));
+#endif
             h[r] = silu * u;
         }
 #pragma omp single

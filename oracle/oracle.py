@@ -20,16 +20,33 @@ SRC = os.path.join(HERE, "moe_oracle.c")
 HDR = os.path.join(HERE, "moe_oracle.h")
 
 
-def build(force: bool = False) -> str:
-    fresh = os.path.exists(SO) and all(
-        os.path.getmtime(SO) >= os.path.getmtime(s) for s in (SRC, HDR))
+# Rounding variants of the oracle (compile-time switches of moe_oracle.c), used
+# only to measure how much the output depends on roundings the pages leave
+# open.  The default oracle is variant "".
+VARIANTS = {
+    "": [],
+    "silu32": ["-DORACLE_SILU_F32"],
+    "muladd": ["-DORACLE_FOLD_MULADD"],
+    "silu32_muladd": ["-DORACLE_SILU_F32", "-DORACLE_FOLD_MULADD"],
+}
+
+
+def so_path(variant: str = "") -> str:
+    return SO if not variant else os.path.join(BUILD, f"liboracle_{variant}.so")
+
+
+def build(force: bool = False, variant: str = "") -> str:
+    so = so_path(variant)
+    fresh = os.path.exists(so) and all(
+        os.path.getmtime(so) >= os.path.getmtime(s) for s in (SRC, HDR))
     if force or not fresh:
         os.makedirs(BUILD, exist_ok=True)
-        tmp = f"{SO}.{os.getpid()}.tmp"
+        tmp = f"{so}.{os.getpid()}.tmp"
         subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
-                               "-fopenmp", "-fPIC", "-shared", SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, SO)
-    return SO
+                               "-fopenmp", "-fPIC", "-shared", *VARIANTS[variant], SRC, "-o", tmp,
+                               "-lm"])
+        os.replace(tmp, so)
+    return so
 
 
 class _Experts(ctypes.Structure):
@@ -39,13 +56,12 @@ class _Experts(ctypes.Structure):
                 ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
 
 
-_lib = None
+_libs = {}
 
 
-def lib() -> ctypes.CDLL:
-    global _lib
-    if _lib is None:
-        L = ctypes.CDLL(build())
+def lib(variant: str = "") -> ctypes.CDLL:
+    if variant not in _libs:
+        L = ctypes.CDLL(build(variant=variant))
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.oracle_bf16_to_f32.restype = f
@@ -67,8 +83,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_combine.argtypes = [vp, vp, vp, i, i, i, vp, vp]
         L.oracle_combine.restype = None
         L.oracle_layer_forward.argtypes = [vp, i, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp]
-        _lib = L
-    return _lib
+        _libs[variant] = L
+    return _libs[variant]
 
 
 def _p(a):
@@ -200,18 +216,18 @@ def unpack(packed, qtype, n):
     return out
 
 
-def qdot(wcodes, w_scale, qa, da):
+def qdot(wcodes, w_scale, qa, da, variant: str = ""):
     wc = _c(wcodes, np.int8)
     qa = _c(qa, np.int8)
     da = _c(da, np.float32)
-    return lib().oracle_qdot(_p(wc), float(w_scale), _p(qa), _p(da), wc.size)
+    return lib(variant).oracle_qdot(_p(wc), float(w_scale), _p(qa), _p(da), wc.size)
 
 
-def expert_token(ex: Experts, e, x_f32, want_h=False):
+def expert_token(ex: Experts, e, x_f32, want_h=False, variant: str = ""):
     x = _c(x_f32, np.float32)
     y = np.empty(ex.H, dtype=np.float32)
     h = np.empty(ex.I, dtype=np.float32) if want_h else None
-    _check(lib().oracle_expert_token(ctypes.byref(ex.struct()), e, _p(x), _p(y), _p(h)),
+    _check(lib(variant).oracle_expert_token(ctypes.byref(ex.struct()), e, _p(x), _p(y), _p(h)),
            "oracle_expert_token")
     return (y, h) if want_h else y
 

@@ -116,6 +116,47 @@ def test_select_matches_brute_force_sort(E, G, TG, K):
     assert np.array_equal(idx, _brute_select(logits, bias, G, TG, K))
 
 
+def _brute_margins(logits, bias, G, TG, K):
+    """Margins at the two selection boundaries from full sorts (fp32 differences):
+    the K-th chosen b minus the best b left among kept groups' experts, and the
+    TG-th kept group score minus the best dropped group score (inf where none is left)."""
+    T, E = logits.shape
+    gsz = E // G
+    ge, gg = np.empty(T, np.float32), np.empty(T, np.float32)
+    for t in range(T):
+        s = np.float32(1.0 / (1.0 + np.exp(-logits[t].astype(np.float64))))
+        b = (s + bias).astype(np.float32)
+        gs = []
+        for g in range(G):
+            vals = sorted(b[g * gsz:(g + 1) * gsz].tolist(), reverse=True)
+            gs.append(np.float32(np.float32(vals[0]) + np.float32(vals[1])))
+        order = sorted(range(G), key=lambda g: (-gs[g], g))
+        gg[t] = np.float32(gs[order[TG - 1]] - gs[order[TG]]) if TG < G else np.float32(np.inf)
+        cand = sorted([e for e in range(E) if e // gsz in order[:TG]], key=lambda e: (-b[e], e))
+        ge[t] = np.float32(b[cand[K - 1]] - b[cand[K]]) if K < len(cand) else np.float32(np.inf)
+    return ge, gg
+
+
+@pytest.mark.parametrize("E,G,TG,K", [(256, 8, 4, 8), (16, 4, 2, 2), (64, 8, 8, 6), (32, 1, 1, 4),
+                                      (8, 2, 1, 4)])
+def test_select_margins_match_brute_force(E, G, TG, K):
+    # the margin diagnostics back the claim that no seeded token sits on a
+    # selection tie; pinned here against full sorts, ties and exhausted
+    # candidate lists included (TG = G: no dropped group; K = group size: no expert left)
+    rng = np.random.default_rng(E * 10 + K + TG)
+    T = 600
+    logits = (1.57 * rng.standard_normal((T, E))).astype(np.float32)
+    logits[: T // 3] = np.round(logits[: T // 3] * 4) / 4
+    for bias in ((0.1 * rng.standard_normal(E)).astype(np.float32), np.zeros(E, np.float32)):
+        _, _, ge, gg = O.select(logits, bias, G, TG, K, 2.5)
+        be, bg = _brute_margins(logits, bias, G, TG, K)
+        assert np.array_equal(ge.view(np.uint32), be.view(np.uint32))
+        assert np.array_equal(gg.view(np.uint32), bg.view(np.uint32))
+        assert np.all(ge >= 0) and np.all(gg >= 0)
+    if K < TG * (E // G):
+        assert np.any(ge[: T // 3] == 0)  # zero bias, quantised logits: exact ties occur
+
+
 def test_select_special_case_is_textbook_topk():
     # one group, no bias: sigmoid is monotone, so the choice is the top-k of the logits
     rng = np.random.default_rng(5)
