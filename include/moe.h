@@ -55,6 +55,11 @@ typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
 /* Human-readable text of an MOE_* code (static string, never NULL). */
 const char* moe_strerror(int code);
 
+/* Text of the CUDA error behind the most recent MOE_ECUDA that a call of this
+ * library returned on the calling thread ("no CUDA error" if none; static
+ * string, never NULL).  This library's own diagnostic, not a step of the layer. */
+const char* moe_cuda_error_string(void);
+
 /* ------------------------------------------------------------ data types */
 
 /* Weight code width.  Layout of one row of n codes (the pages name packed

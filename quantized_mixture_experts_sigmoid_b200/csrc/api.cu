@@ -85,7 +85,14 @@ int check_experts(const moe_experts* ex) {
     return MOE_OK;
 }
 
-int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+// The CUDA error behind the most recent MOE_ECUDA returned on this thread.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+int cuda_rc(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    g_last_cuda_error = e;
+    return MOE_ECUDA;
+}
 
 struct LayerWs {
     int32_t* status;
@@ -246,6 +253,10 @@ const char* moe_strerror(int code) {
         case MOE_ETOO_LARGE: return "batch exceeds the fixed scratch capacity of moe_route_noalloc";
         default: return "unknown moe error code";
     }
+}
+
+const char* moe_cuda_error_string(void) {
+    return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
 }
 
 size_t moe_route_workspace_bytes(int T, const moe_router_cfg* cfg) {

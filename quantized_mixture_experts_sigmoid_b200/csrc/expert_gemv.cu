@@ -5,13 +5,18 @@
 // dequant-on-use, an integer-dot kernel against Q8_0 int8 activations, and
 // batch-union MoE (each distinct expert applied to all its positions).
 //
-// up/gate kernel: one CTA per (32-row block of h, distinct expert).  It
-// stages the Q8_0 activations of up to TC of the expert's tokens in shared
-// memory, streams the 32 gate rows and 32 up rows (integer dot per block,
-// fp32 promotion), applies SwiGLU and quantises the 32 h values of each token
-// to one Q8_0 block, written by pair index.
-// down kernel: one CTA per (32 output rows, distinct expert); it streams the
-// rows against the staged Q8_0(h) of the expert's pairs and writes y by
+// Every weight row is consumed by one lane, which folds the row's 32-code
+// blocks in ascending order with one fp32 fused multiply-add per block: the
+// quantised dot of the layer's definition, bit for bit (a one-ulp difference in
+// h could flip a Q8_0 code of h).
+//
+// up/gate kernel: one CTA per (32-row block of h, distinct expert).  It stages
+// the Q8_0 activations of up to kUgTok of the expert's tokens in shared
+// memory; warp w takes the gate (w even) or up (w odd) rows, lane r row r, for
+// the tokens of group w / 2; then SwiGLU and Q8_0 of the 32 h values of each
+// token give one Q8_0 block, written by pair index.
+// down kernel: one CTA per (32 output rows, distinct expert); warp w takes
+// kDownTpw of the expert's staged pairs, lane r output row r; y is written by
 // (token, slot).
 #include "common.cuh"
 #include "kernels.cuh"
@@ -22,10 +27,12 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUgRows = 32;    // h rows per up/gate CTA
-constexpr int kDownRows = 32;  // output rows per down CTA
-constexpr int kUgTok = 8;      // tokens staged per pass (up/gate)
-constexpr int kDownTok = 16;   // pairs staged per pass (down)
+constexpr int kUgRows = 32;                     // h rows per up/gate CTA
+constexpr int kDownRows = 32;                   // output rows per down CTA
+constexpr int kUgTpw = 2;                       // tokens per warp (up/gate)
+constexpr int kUgTok = kUgTpw * kWarps / 2;     // tokens staged per pass (up/gate): 8
+constexpr int kDownTpw = 2;                     // pairs per warp (down)
+constexpr int kDownTok = kDownTpw * kWarps;     // pairs staged per pass (down): 16
 
 struct ExpertRange {
     int e, p0, p1;
@@ -45,7 +52,29 @@ __device__ __forceinline__ bool expert_range(const UnionView& un, int u, int T, 
     return true;
 }
 
-template <int QT, int TC>
+// Lane-per-row quantised dots of one weight row against TPW staged activation
+// rows (t0 .. t0 + nt - 1 of the staging area): blocks ascending, one fused
+// multiply-add per block; returns the unscaled sums.
+template <int QT, int TPW>
+__device__ __forceinline__ void row_dots(const uint8_t* row, int nb, const uint4* a0, const uint4* a1,
+                                         const float* ad, const int32_t* as, int t0, int nt,
+                                         float (&acc)[TPW]) {
+#pragma unroll
+    for (int t = 0; t < TPW; ++t) acc[t] = 0.0f;
+#pragma unroll 4
+    for (int b = 0; b < nb; ++b) {
+        const WBlock<QT> w = load_wblock_l1<QT>(row, b);
+#pragma unroll
+        for (int t = 0; t < TPW; ++t) {
+            if (t < nt) {
+                const int q = (t0 + t) * nb + b;
+                acc[t] = fmaf(static_cast<float>(block_dot<QT>(w, a0[q], a1[q], as[q])), ad[q], acc[t]);
+            }
+        }
+    }
+}
+
+template <int QT>
 __global__ void __launch_bounds__(kThreads)
 k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
           const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I,
@@ -54,24 +83,25 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = H / 32;
     uint4* a0 = reinterpret_cast<uint4*>(smem);
-    uint4* a1 = a0 + TC * nb;
-    float* ad = reinterpret_cast<float*>(a1 + TC * nb);
-    int32_t* as = reinterpret_cast<int32_t*>(ad + TC * nb);
-    float* gbuf = reinterpret_cast<float*>(as + TC * nb);
-    float* ubuf = gbuf + TC * kUgRows;
+    uint4* a1 = a0 + kUgTok * nb;
+    float* ad = reinterpret_cast<float*>(a1 + kUgTok * nb);
+    int32_t* as = reinterpret_cast<int32_t*>(ad + kUgTok * nb);
+    float* gbuf = reinterpret_cast<float*>(as + kUgTok * nb);
+    float* ubuf = gbuf + kUgTok * kUgRows;
 
     ExpertRange er;
     if (!expert_range(un, blockIdx.y, T, er)) return;
     const int r0 = blockIdx.x * kUgRows;
     const size_t rb = static_cast<size_t>(H) * QT / 8;
-    const uint8_t* Wg = w_gate + (static_cast<size_t>(er.e) * I + r0) * rb;
-    const uint8_t* Wu = w_up + (static_cast<size_t>(er.e) * I + r0) * rb;
-    const float* sg = s_gate + static_cast<size_t>(er.e) * I + r0;
-    const float* su = s_up + static_cast<size_t>(er.e) * I + r0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m = warp & 1, tg = warp >> 1;  // gate / up rows; token group
+    const size_t row = static_cast<size_t>(er.e) * I + r0 + lane;
+    const uint8_t* wrow = (m == 0 ? w_gate : w_up) + row * rb;
+    const float srow = __ldg((m == 0 ? s_gate : s_up) + row);
+    float* dst = m == 0 ? gbuf : ubuf;
 
-    for (int pc = er.p0; pc < er.p1; pc += TC) {
-        const int nt = min(TC, er.p1 - pc);
+    for (int pc = er.p0; pc < er.p1; pc += kUgTok) {
+        const int nt = min(kUgTok, er.p1 - pc);
         for (int i = 0; i < nt; ++i) {
             const int tok = un.uniq ? un.pair_tok[pc + i] : pc + i;
             stage_act_row<QT>(qx + static_cast<size_t>(tok) * H, dx + static_cast<size_t>(tok) * nb,
@@ -79,35 +109,13 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
                               kThreads);
         }
         __syncthreads();
-        for (int j = warp; j < 2 * kUgRows; j += kWarps) {
-            const uint8_t* row = j < kUgRows ? Wg + j * rb : Wu + (j - kUgRows) * rb;
-            float acc[TC];
+        const int t0 = tg * kUgTpw, ntw = min(kUgTpw, nt - t0);
+        if (ntw > 0) {
+            float acc[kUgTpw];
+            row_dots<QT, kUgTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, acc);
 #pragma unroll
-            for (int t = 0; t < TC; ++t) acc[t] = 0.0f;
-#pragma unroll 2
-            for (int b = lane; b < nb; b += 32) {
-                const WBlock<QT> w = load_wblock<QT>(row, b);
-#pragma unroll
-                for (int t = 0; t < TC; ++t) {
-                    if (t < nt) {
-                        const int isum = block_dot<QT>(w, a0[t * nb + b], a1[t * nb + b], as[t * nb + b]);
-                        acc[t] = fmaf(static_cast<float>(isum), ad[t * nb + b], acc[t]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < TC; ++t) {
-                if (t < nt) {
-                    const float v = warp_sum_f32(acc[t]);
-                    if (lane == 0) {
-                        if (j < kUgRows) {
-                            gbuf[t * kUgRows + j] = __fmul_rn(v, sg[j]);
-                        } else {
-                            ubuf[t * kUgRows + j - kUgRows] = __fmul_rn(v, su[j - kUgRows]);
-                        }
-                    }
-                }
-            }
+            for (int t = 0; t < kUgTpw; ++t)
+                if (t < ntw) dst[(t0 + t) * kUgRows + lane] = __fmul_rn(acc[t], srow);
         }
         __syncthreads();
         for (int t = warp; t < nt; t += kWarps) {
@@ -122,7 +130,7 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     }
 }
 
-template <int QT, int TC>
+template <int QT>
 __global__ void __launch_bounds__(kThreads)
 k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
@@ -130,52 +138,38 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = I / 32;
     uint4* a0 = reinterpret_cast<uint4*>(smem);
-    uint4* a1 = a0 + TC * nb;
-    float* ad = reinterpret_cast<float*>(a1 + TC * nb);
-    int32_t* as = reinterpret_cast<int32_t*>(ad + TC * nb);
+    uint4* a1 = a0 + kDownTok * nb;
+    float* ad = reinterpret_cast<float*>(a1 + kDownTok * nb);
+    int32_t* as = reinterpret_cast<int32_t*>(ad + kDownTok * nb);
 
     ExpertRange er;
     if (!expert_range(un, blockIdx.y, T, er)) return;
     const int c0 = blockIdx.x * kDownRows;
     const size_t rb = static_cast<size_t>(I) * QT / 8;
-    const uint8_t* Wd = w_down + (static_cast<size_t>(er.e) * H + c0) * rb;
-    const float* sd = s_down + static_cast<size_t>(er.e) * H + c0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const size_t row = static_cast<size_t>(er.e) * H + c0 + lane;
+    const uint8_t* wrow = w_down + row * rb;
+    const float srow = __ldg(s_down + row);
 
-    for (int pc = er.p0; pc < er.p1; pc += TC) {
-        const int nt = min(TC, er.p1 - pc);
+    for (int pc = er.p0; pc < er.p1; pc += kDownTok) {
+        const int nt = min(kDownTok, er.p1 - pc);
         for (int i = 0; i < nt; ++i) {
             const size_t p = static_cast<size_t>(pc + i);
             stage_act_row<QT>(qh + p * I, dh + p * nb, nb, a0 + i * nb, a1 + i * nb, ad + i * nb,
                               as + i * nb, threadIdx.x, kThreads);
         }
         __syncthreads();
-        for (int j = warp; j < kDownRows; j += kWarps) {
-            const uint8_t* row = Wd + j * rb;
-            float acc[TC];
+        const int t0 = warp * kDownTpw, ntw = min(kDownTpw, nt - t0);
+        if (ntw > 0) {
+            float acc[kDownTpw];
+            row_dots<QT, kDownTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, acc);
 #pragma unroll
-            for (int t = 0; t < TC; ++t) acc[t] = 0.0f;
-#pragma unroll 2
-            for (int b = lane; b < nb; b += 32) {
-                const WBlock<QT> w = load_wblock<QT>(row, b);
-#pragma unroll
-                for (int t = 0; t < TC; ++t) {
-                    if (t < nt) {
-                        const int isum = block_dot<QT>(w, a0[t * nb + b], a1[t * nb + b], as[t * nb + b]);
-                        acc[t] = fmaf(static_cast<float>(isum), ad[t * nb + b], acc[t]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < TC; ++t) {
-                if (t < nt) {
-                    const float v = warp_sum_f32(acc[t]);
-                    if (lane == 0) {
-                        const int p = pc + t;
-                        const int tok = un.uniq ? un.pair_tok[p] : p;
-                        const int slot = un.uniq ? un.pair_slot[p] : 0;
-                        y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + j] = __fmul_rn(v, sd[j]);
-                    }
+            for (int t = 0; t < kDownTpw; ++t) {
+                if (t < ntw) {
+                    const int p = pc + t0 + t;
+                    const int tok = un.uniq ? un.pair_tok[p] : p;
+                    const int slot = un.uniq ? un.pair_slot[p] : 0;
+                    y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + lane] = __fmul_rn(acc[t], srow);
                 }
             }
         }
@@ -188,7 +182,7 @@ cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx,
                        const UnionView& un, int8_t* qh, float* dh, cudaStream_t st) {
     const int nb = ex.hidden / 32;
     const size_t smem = static_cast<size_t>(kUgTok) * nb * 40 + 2 * kUgTok * kUgRows * sizeof(float);
-    auto kern = k_up_gate<QT, kUgTok>;
+    auto kern = k_up_gate<QT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(ex.inter / kUgRows, un.max_unique);
@@ -202,7 +196,7 @@ cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, in
                     const UnionView& un, float* y, cudaStream_t st) {
     const int nb = ex.inter / 32;
     const size_t smem = static_cast<size_t>(kDownTok) * nb * 40;
-    auto kern = k_down<QT, kDownTok>;
+    auto kern = k_down<QT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(ex.hidden / kDownRows, un.max_unique);

@@ -21,36 +21,22 @@ struct WBlock {
     uint32_t w[QT];
 };
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-    uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-        : "l"(p));
-    return r;
-}
-
-__device__ __forceinline__ uint2 ld_stream_v2(const void* p) {
-    uint2 r;
-    asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-    return r;
-}
-
+// Block b of a weight row through the L1 cache (lane-per-row kernels: a lane
+// reads its row's consecutive blocks, so the rest of each 32-byte sector is
+// reused).
 template <int QT>
-__device__ __forceinline__ WBlock<QT> load_wblock(const uint8_t* row, int b) {
+__device__ __forceinline__ WBlock<QT> load_wblock_l1(const uint8_t* row, int b) {
     WBlock<QT> r;
     if constexpr (QT == 2) {
-        const uint2 v = ld_stream_v2(row + 8 * b);
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(row + 8 * b));
         r.w[0] = v.x;
         r.w[1] = v.y;
     } else if constexpr (QT == 4) {
-        const uint4 v = ld_stream_v4(row + 16 * b);
-        r.w[0] = v.x;
-        r.w[1] = v.y;
-        r.w[2] = v.z;
-        r.w[3] = v.w;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + 16 * b));
+        r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
     } else {
-        const uint4 v0 = ld_stream_v4(row + 32 * b);
-        const uint4 v1 = ld_stream_v4(row + 32 * b + 16);
+        const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(row + 32 * b));
+        const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(row + 32 * b + 16));
         r.w[0] = v0.x; r.w[1] = v0.y; r.w[2] = v0.z; r.w[3] = v0.w;
         r.w[4] = v1.x; r.w[5] = v1.y; r.w[6] = v1.z; r.w[7] = v1.w;
     }

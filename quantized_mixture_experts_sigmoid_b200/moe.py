@@ -30,7 +30,8 @@ MOE_OUT_BF16, MOE_OUT_F32 = 0, 1
 
 class MoeError(RuntimeError):
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn} failed: {code} ({strerror(code)})")
+        extra = f": {lib().moe_cuda_error_string().decode()}" if code == MOE_ECUDA else ""
+        super().__init__(f"{fn} failed: {code} ({strerror(code)}{extra})")
         self.code = code
 
 
@@ -88,7 +89,7 @@ EXPORTS = ["moe_strerror", "moe_route_workspace_bytes", "moe_route", "moe_union"
            "moe_quantize_q8_0", "moe_expert_ffn_workspace_bytes", "moe_expert_ffn_q",
            "moe_combine", "moe_layer_workspace_bytes", "moe_layer_forward",
            "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count",
-           "moe_route_noalloc", "moe_layer_path"]
+           "moe_route_noalloc", "moe_layer_path", "moe_cuda_error_string"]
 
 
 def lib() -> ctypes.CDLL:
@@ -103,6 +104,8 @@ def lib() -> ctypes.CDLL:
     vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     L.moe_strerror.argtypes = [i]
     L.moe_strerror.restype = ctypes.c_char_p
+    L.moe_cuda_error_string.argtypes = []
+    L.moe_cuda_error_string.restype = ctypes.c_char_p
     L.moe_route_workspace_bytes.argtypes = [i, vp]
     L.moe_route_workspace_bytes.restype = sz
     L.moe_route.argtypes = [vp, i, i, vp, vp, vp, vp, vp, vp, sz, vp]

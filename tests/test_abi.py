@@ -31,8 +31,10 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_error_strings():
-    for code in (0, -1, -2, -3, -4, -5, -6, -99):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -99):
         assert isinstance(moe.strerror(code), str) and moe.strerror(code)
+    # no call on this thread has returned MOE_ECUDA: the CUDA error text says so
+    assert moe.lib().moe_cuda_error_string().decode() == "no CUDA error"
 
 
 P = 1 << 20  # a fake, 16-byte aligned "device" address: never dereferenced on these paths
