@@ -51,6 +51,40 @@ def _experts(sh, ids, shared=False):
     return ex
 
 
+def layer_outputs(sh, batches, variant: str = ""):
+    """Oracle layer outputs of each batch (a list of token ids, one layer call
+    each): [(x_bits, idx, w, out_f32)], with each touched expert generated once
+    and evaluated for all its tokens (so no more than one expert is held)."""
+    W, b = synth.router_weight(sh), synth.router_bias(sh)
+    xbits, xs, routes = [], [], []
+    for tok in batches:
+        x = synth.hidden_states(sh, tokens=tok)
+        idx, w, _, _ = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+        xbits.append(x)
+        xs.append(synth.bf16_to_f32(x).astype(np.float32))
+        routes.append((idx, w))
+    by_expert = defaultdict(list)
+    for bi, (idx, _) in enumerate(routes):
+        for t in range(idx.shape[0]):
+            for k in range(idx.shape[1]):
+                by_expert[int(idx[t, k])].append((bi, t, k))
+    y = {}
+    units = [(e, by_expert[e]) for e in sorted(by_expert)]
+    units.append((-1, [(bi, t, -1) for bi, x in enumerate(xs) for t in range(x.shape[0])]))
+    for e, uses in units:
+        ex = _experts(sh, [0], shared=True) if e < 0 else _experts(sh, [e])
+        for bi, t, k in uses:
+            y[(bi, t, k)] = O.expert_token(ex, 0 if e < 0 else e, xs[bi][t], variant=variant)
+    out = []
+    for bi, (idx, w) in enumerate(routes):
+        T, K = idx.shape
+        yp = np.stack([np.stack([y[(bi, t, k)] for k in range(K)]) for t in range(T)])
+        ys = np.stack([y[(bi, t, -1)] for t in range(T)])
+        of, _ = O.combine(yp, w, ys)
+        out.append((xbits[bi], idx, w, of))
+    return out
+
+
 def rel_metric(got, ref):
     got = np.asarray(got, np.float64).reshape(-1, ref.shape[-1])
     ref = np.asarray(ref, np.float64).reshape(-1, ref.shape[-1])

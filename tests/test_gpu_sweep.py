@@ -1,0 +1,114 @@
+"""Parity beyond one seed: many seeded tokens through the small-batch layer on
+the GPU, each compared with the oracle element by element, and routing ties
+resolved by the lower index on every routing kernel.
+
+Decode: 256 distinct tokens, one layer call each (T = 1).  MTP verify: 64
+calls of 4 correlated positions (256 positions); each call's batch union must
+hold 8 to 32 distinct experts, as the workload prescribes.  The oracle
+evaluates each touched expert once for all its tokens.  The largest error and
+the number of tokens whose error suggests a flipped Q8_0(h) code (above 1e-4)
+are printed; the bar is the same 2e-3 as everywhere.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import oracle as O
+from oracle.variant_report import layer_outputs
+from quantized_mixture_experts_sigmoid_b200 import moe
+from tests.gpu_fixtures import device_layer, to_dev_bf16
+from tests.helpers import rel_err_rows
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+def _sweep(sh, batches):
+    dev = device_layer(sh)
+    assert moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"]) == moe.PATH_FUSED
+    ref = layer_outputs(sh, batches)
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
+    errs, us = [], []
+    for x, idx_o, w_o, of_o in ref:
+        T = x.shape[0]
+        out = torch.empty(T, sh.H, dtype=torch.float32, device="cuda")
+        idx = torch.empty(T, sh.top_k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, sh.top_k, dtype=torch.float32, device="cuda")
+        moe.moe_layer_forward(to_dev_bf16(x), dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"],
+                              out, ws, idx, w)
+        assert np.array_equal(idx.cpu().numpy(), idx_o)
+        assert np.array_equal(w.cpu().numpy().view(np.uint32), w_o.view(np.uint32))
+        og = out.cpu().numpy()
+        errs += [rel_err_rows(og[t:t + 1], of_o[t:t + 1]) for t in range(T)]
+        us.append(len(np.unique(idx_o)))
+    assert moe.moe_workspace_status(ws) == 0
+    errs = np.array(errs)
+    print(f"\n{sh.name}: {errs.size} tokens, max rel err {errs.max():.3e}, "
+          f"tokens above 1e-4: {int(np.sum(errs > 1e-4))}, distinct experts per call {min(us)}..{max(us)}")
+    assert errs.max() <= TOL, errs.max()
+    return us
+
+
+def test_decode_sweep_256_tokens():
+    sh = synth.CONFIGS["decode"]
+    _sweep(sh, [[t] for t in range(1000, 1256)])
+
+
+def test_verify_sweep_64_calls():
+    sh = synth.CONFIGS["verify"]
+    us = _sweep(sh, [list(range(4 * i + 1000, 4 * i + 1004)) for i in range(64)])
+    assert min(us) >= 8 and max(us) <= 32
+
+
+def _tie_router(sh):
+    """Router weights and bias with exact ties.  Groups 0-2 carry a large bias so they are
+    always kept; groups 3 and 6 are copies of each other (equal group scores for every
+    token) competing for the last kept group; nine experts of the kept groups share one
+    weight row and bias and outrank everything else, competing for the eight slots."""
+    W = synth.router_weight(sh).copy()
+    b = synth.router_bias(sh).copy()
+    gs = sh.E // sh.n_group
+    b[: 3 * gs] += 2.0
+    b[3 * gs: 4 * gs] += 1.0
+    W[6 * gs: 7 * gs] = W[3 * gs: 4 * gs]
+    b[6 * gs: 7 * gs] = b[3 * gs: 4 * gs]
+    tied = [5, 6, 20, 37, 38, 69, 70, 90, 91]
+    W[tied] = W[tied[0]]
+    b[tied] = 3.0
+    return W, b, tied
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_routing_ties_lower_index_on_every_kernel(T):
+    sh = synth.CONFIGS["decode"].with_(T=T)
+    W, b, tied = _tie_router(sh)
+    x = synth.hidden_states(sh, tokens=range(T))
+    idx_o, w_o, gap_e, gap_g = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+    # the construction does produce ties at both boundaries, and the lower index wins
+    assert np.all(gap_e == 0) and np.all(gap_g == 0)
+    assert all(sorted(r.tolist()) == tied[:8] for r in idx_o)
+    Wd, bd = torch.from_numpy(W).cuda(), torch.from_numpy(b).cuda()
+    cfg = moe.RouterCfg(sh.E, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+    xd = to_dev_bf16(x)
+    for route in ("moe_route", "moe_route_noalloc"):
+        idx = torch.empty(T, sh.top_k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, sh.top_k, dtype=torch.float32, device="cuda")
+        if route == "moe_route":
+            moe.moe_route(xd, Wd, bd, cfg, idx, w, moe.workspace(moe.moe_route_workspace_bytes(T, cfg)))
+        else:
+            moe.moe_route_noalloc(xd, Wd, bd, cfg, idx, w)
+        assert np.array_equal(idx.cpu().numpy(), idx_o), route
+        assert np.array_equal(w.cpu().numpy().view(np.uint32), w_o.view(np.uint32)), route
+    # the fused layer kernel routes in its own warp
+    dev = device_layer(synth.CONFIGS["decode"])
+    assert moe.moe_layer_path(T, cfg, dev["routed"], dev["shared"]) == moe.PATH_FUSED
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(T, cfg, dev["routed"], dev["shared"]))
+    out = torch.empty(T, sh.H, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, sh.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, sh.top_k, dtype=torch.float32, device="cuda")
+    moe.moe_layer_forward(xd, Wd, bd, cfg, dev["routed"], dev["shared"], out, ws, idx, w)
+    assert moe.moe_workspace_status(ws) == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_o)
+    assert np.array_equal(w.cpu().numpy().view(np.uint32), w_o.view(np.uint32))

@@ -20,7 +20,7 @@ from tests.helpers import layer_inputs, oracle_experts, rel_err_rows
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
-SAMPLE = 12
+SAMPLE = 64
 
 
 def test_prefill_full_size_sampled():
