@@ -65,21 +65,26 @@ KERNEL_SOURCES = ("decode_fused.cu", "common.cuh", "quant.cuh", "sm100_async.cuh
 
 
 def profiled_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary, or None when
-    the kernel sources have changed since that capture."""
+    """DRAM bytes per launch of the fused kernel from the committed ncu capture
+    (profiles/k_decode_fused_decode.json), or None when the kernel sources have
+    changed since that capture."""
     import hashlib
-    import re
     try:
-        txt = open(os.path.join(ROOT, "profiles", "k_decode_fused_decode.md")).read()
-        traffic = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt).group(1))
-        sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt).group(1)
-    except (OSError, AttributeError):
+        with open(os.path.join(ROOT, "profiles", "k_decode_fused_decode.json")) as fh:
+            rec = json.load(fh)
+        traffic, sha = int(rec["traffic_bytes_per_launch"]), rec["source_sha256"]
+    except (OSError, KeyError, ValueError):
         return None
+    return traffic if kernel_sources_sha256() == sha else None
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "quantized_mixture_experts_sigmoid_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    return traffic if h.hexdigest() == sha else None
+    return h.hexdigest()
 
 
 def parse():
@@ -97,6 +102,11 @@ def parse():
     ap.add_argument("--prefill-tokens", type=int, default=2048, help="prefill batch size (profiling: smaller)")
     ap.add_argument("--prefill-experts", type=int, default=256,
                     help="routed experts of the prefill layer (profiling: 32, in 4 groups)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the verify and stacked entries (measured only on one GPU)")
+    ap.add_argument("--clock-window", type=float, default=1.5,
+                    help="seconds of the same decode loop, right after the timed steps, during which "
+                         "clocks are sampled")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill measurement and print its entry (for profiler captures)")
     return ap.parse_args()
@@ -106,7 +116,7 @@ def parse():
 def oracle_sample(sh, seconds: float, first_token: int = 0, max_tokens: int | None = None):
     """Time the CPU oracle's full layer on successive seeded tokens for ~`seconds`."""
     from oracle import oracle as O
-    from tests.helpers import oracle_experts
+    from oracle.synth_inputs import oracle_experts
 
     W = synth.router_weight(sh)
     b = synth.router_bias(sh)
@@ -149,51 +159,68 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- clocks
+# NVML clock-event reason bits (nvmlClocksEventReason*)
+_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown"}
+
+
 class ClockSampler:
-    def __init__(self, gpu: int):
-        self.gpu = gpu
-        self.proc = None
+    """SM clock and clock-event reasons sampled every `period` seconds in a thread
+    (NVML, in process); mark() labels the samples taken from then on."""
+
+    def __init__(self, gpu: int, period: float = 0.002):
+        self.gpu, self.period = gpu, period
+        self.samples = []  # (label, sm_mhz, max_mhz, reasons bitmask)
+        self.label = None
+        self._stop = None
 
     def __enter__(self):
-        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    if self.label is not None:
+                        self.samples.append((self.label, sm, mx, rs))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
-    def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+    def mark(self, label):
+        self.label = label
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
+    def __exit__(self, *a):
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+
+    def summary(self, labels):
+        sel = [x for x in self.samples if x[0] in labels]
+        reasons = set()
+        for _, _, _, rs in sel:
+            for bit, nm in _REASONS.items():
+                if rs & bit:
                     reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median([x[1] for x in sel]) if sel else None,
+               "sm_max_mhz": sel[0][2] if sel else None, "reasons": sorted(reasons),
+               "samples": len(sel), "period_ms": self.period * 1e3}
+        for lb in labels:
+            out[f"samples_{lb}"] = sum(1 for x in sel if x[0] == lb)
+        return out
 
 
 # ---------------------------------------------------------------- CUDA arm
@@ -300,12 +327,126 @@ def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     }
 
 
+def verify_measurement(moe, L, device_layer, to_dev_bf16, name: str, n_layers: int = 4, steps: int = 200):
+    """MTP verify (T = 4 correlated positions, the fused kernel): tokens/s, the realised batch
+    unions, and the fused kernel's bytes per call against the HBM roofline."""
+    import ctypes
+
+    import torch
+    sh = synth.CONFIGS[name]
+    devs = [device_layer(sh, layer=l) for l in range(n_layers)]
+    T, K = sh.T, sh.top_k
+    n_calls = 64
+    pool = to_dev_bf16(synth.hidden_states(sh, tokens=range(T * n_calls)))
+    out = torch.empty(T, sh.H, dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty(steps, T, K, dtype=torch.int32, device="cuda")
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(T, devs[0]["cfg"], devs[0]["routed"], devs[0]["shared"]))
+    path = moe.moe_layer_path(T, devs[0]["cfg"], devs[0]["routed"], devs[0]["shared"])
+
+    def step(i):
+        d = devs[i % n_layers]
+        j = (i % n_calls) * T
+        moe.moe_layer_forward(pool[j:j + T], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], out, ws,
+                              idx[i % steps])
+
+    for i in range(5):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    L.moe_profile_enable(1)
+    for i in range(steps):
+        step(i)
+    torch.cuda.synchronize()
+    kms, kn = ctypes.c_double(0), ctypes.c_int(0)
+    L.moe_profile_read(ctypes.byref(kms), ctypes.byref(kn))
+    L.moe_profile_enable(0)
+    if moe.moe_workspace_status(ws) != 0:
+        raise RuntimeError(f"device status error during the {name} measurement")
+    ids = idx.cpu().numpy()
+    U = np.array([len(np.unique(ids[i])) for i in range(steps)])
+    call_bytes = (U.mean() + 1) * sh.expert_bytes() + sh.router_bytes()
+    k_ms = kms.value / max(kn.value, 1)
+    hbm, kind = peaks()
+    del devs, ws
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"MTP verify batch union: T={T} correlated positions, GLM-5.2 layer shape, "
+                    f"{'int8' if sh.qtype == 8 else 'int4'} experts, {n_layers} resident layers rotated",
+        "path": {moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core", moe.PATH_GENERAL: "general"}[path],
+        "tokens_per_s": T / (ms / 1e3), "ms_per_call": ms,
+        "distinct_experts": {"mean": float(U.mean()), "min": int(U.min()), "max": int(U.max())},
+        "bytes_per_call": call_bytes, "GBps": call_bytes / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "k_decode_fused", "achieved": call_bytes / (k_ms / 1e3) / 1e9,
+                     "peak": hbm, "peak_kind": kind, "unit": "GB/s",
+                     "frac": call_bytes / (k_ms / 1e3) / 1e9 / hbm, "ms_per_launch": k_ms},
+    }
+
+
+def stacked_measurement(moe, device_layer, to_dev_bf16, name: str, Ts, reps: int = 10):
+    """Stacked decode: all 16 layers resident, timed as one sequence of 16 layer calls (a token
+    through the stack), fresh seeded hidden states per layer."""
+    import torch
+    sh = synth.CONFIGS[name]
+    layers = [device_layer(sh, layer=l) for l in range(sh.n_layers)]
+    entries = []
+    for T in Ts:
+        shT = sh.with_(T=T)
+        xs = [to_dev_bf16(synth.hidden_states(shT, layer=l)) for l in range(sh.n_layers)]
+        d0 = layers[0]
+        ws = moe.workspace(moe.moe_layer_workspace_bytes(T, d0["cfg"], d0["routed"], d0["shared"]))
+        out = torch.empty(T, sh.H, dtype=torch.bfloat16, device="cuda")
+        idx = torch.empty(sh.n_layers, T, sh.top_k, dtype=torch.int32, device="cuda")
+        path = moe.moe_layer_path(T, d0["cfg"], d0["routed"], d0["shared"])
+
+        def sequence():
+            for l in range(sh.n_layers):
+                d = layers[l]
+                moe.moe_layer_forward(xs[l], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], out, ws,
+                                      idx[l])
+
+        sequence()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            sequence()
+        e1.record()
+        torch.cuda.synchronize()
+        if moe.moe_workspace_status(ws) != 0:
+            raise RuntimeError(f"device status error during the {name} T={T} measurement")
+        ms = e0.elapsed_time(e1) / reps
+        ids = idx.cpu().numpy()
+        U = np.array([len(np.unique(ids[l])) for l in range(sh.n_layers)])
+        seq_bytes = float(((U + 1) * sh.expert_bytes() + sh.router_bytes()).sum())
+        hbm, kind = peaks()
+        entries.append({
+            "workload": f"stacked decode: {sh.n_layers} resident GLM-5.2 layers "
+                        f"({sh.n_layers * (sh.E + 1) * sh.expert_bytes() / 1e9:.1f} GB "
+                        f"{'int2' if sh.qtype == 2 else 'int4'}), T={T}, one sequence of {sh.n_layers} layer calls",
+            "path": {moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core", moe.PATH_GENERAL: "general"}[path],
+            "tokens_per_s": T / (ms / 1e3), "ms_per_sequence": ms, "layer_calls_per_s": sh.n_layers / (ms / 1e3),
+            "distinct_experts_per_layer": float(U.mean()), "bytes_per_sequence": seq_bytes,
+            "GBps": seq_bytes / (ms / 1e3) / 1e9, "frac_of_hbm_peak": seq_bytes / (ms / 1e3) / 1e9 / hbm,
+            "peak_kind": kind,
+        })
+        del ws, xs
+    del layers
+    torch.cuda.empty_cache()
+    return entries
+
+
 def run_cuda(args):
     import torch
     import torch.distributed as dist
 
     from quantized_mixture_experts_sigmoid_b200 import moe
-    from tests.gpu_fixtures import device_layer, to_dev_bf16
+    from synth.device import device_layer, to_dev_bf16
 
     if args.prefill_only:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
@@ -337,6 +478,7 @@ def run_cuda(args):
         moe.moe_layer_forward(xs[j:j + 1], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], out, ws,
                               idx, wts)
 
+    clk = ClockSampler(local).__enter__()
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -351,23 +493,42 @@ def run_cuda(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        wall0 = time.perf_counter()
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i)
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        wall = time.perf_counter() - wall0
+    clk.mark("timed")
+    wall0 = time.perf_counter()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clk.mark(None)
     launches = L.moe_launch_count() - launches0
     dev_ms = ev0.elapsed_time(ev1)
     dev_ms = max_over_ranks(dev_ms, world, "cuda")
     if moe.moe_workspace_status(ws) != 0:
         raise RuntimeError("device status error during timing")
 
+    # ---- clock window: the same back-to-back loop for at least `clock_window` seconds
+    # right after the timed steps (which last about a millisecond at the driver's K, too
+    # short to sample); its own tokens/s is reported next to the timed value
+    clk.mark("window")
+    cw_steps, cw_wall0 = 0, time.perf_counter()
+    cw0, cw1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cw0.record(stream)
+    while time.perf_counter() - cw_wall0 < args.clock_window:
+        for i in range(500):
+            step(args.warmup + args.steps + cw_steps + i)
+        cw_steps += 500
+        torch.cuda.synchronize()
+    cw1.record(stream)
+    torch.cuda.synchronize()
+    clk.mark(None)
+    cw_ms = cw0.elapsed_time(cw1)
+    clk.__exit__(None, None, None)
+
     # ---- the dominant kernel's own duration: events around each launch (they also keep
     # consecutive launches from overlapping, so this is the standalone kernel time)
-    prof_steps = min(args.steps, 2000)
+    prof_steps = min(args.steps, 2000) if args.steps >= 200 else 2000
     torch.cuda.synchronize()
     L.moe_profile_enable(1)
     for i in range(prof_steps):
@@ -381,7 +542,7 @@ def run_cuda(args):
     x_host = torch.from_numpy(pool.view(np.int16)).view(torch.bfloat16).pin_memory()
     out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    e2e_steps = min(args.steps, 3000)
+    e2e_steps = max(min(args.steps, 3000), 1000)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -397,7 +558,15 @@ def run_cuda(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, world, "cuda")
+    del devs, ws
+    torch.cuda.empty_cache()
 
+    extras = {}
+    if world == 1 and not args.no_extras:
+        extras["verify"] = verify_measurement(moe, L, device_layer, to_dev_bf16, "verify")
+        extras["verify_int8"] = verify_measurement(moe, L, device_layer, to_dev_bf16, "verify_int8")
+        extras["stacked"] = stacked_measurement(moe, device_layer, to_dev_bf16, "stacked", (1, 8))
+        extras["stacked_int2"] = stacked_measurement(moe, device_layer, to_dev_bf16, "stacked_int2", (1,))
     prefill = prefill_measurement(args, moe, L, device_layer, to_dev_bf16) if args.prefill else None
 
     if world > 1:
@@ -417,6 +586,9 @@ def run_cuda(args):
     dom_bytes = layer_bytes
     dom_ms = kms.value / max(kn.value, 1)
     dom_gbs = dom_bytes / (dom_ms / 1e3) / 1e9 if dom_ms > 0 else None
+    clocks = clk.summary(("timed", "window"))
+    clocks["window_s"] = cw_ms / 1e3
+    clocks["window_tokens_per_s"] = T * cw_steps / (cw_ms / 1e3)
     line = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -436,11 +608,12 @@ def run_cuda(args):
                      "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": profiled_traffic(),
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
         "e2e": {"value": replicas_tokens_per_s(world, T, e2e_steps, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2},
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps},
         "gpu_launches": int(launches),
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "wall_s_timed_region": wall,
     }
+    line.update(extras)
     if prefill is not None:
         line["prefill"] = prefill
     if not args.no_cpu_baseline and world == 1:

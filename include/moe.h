@@ -123,6 +123,9 @@ size_t moe_route_workspace_bytes(int T, const moe_router_cfg* cfg);
  *   topk_w[t][k] = s[idx] / sum_k s[idx] * routed_scaling_factor
  * x: [T][H] bf16; w_router: [E][H] fp32; bias: [E] fp32;
  * topk_idx: [T][top_k] int32 out; topk_w: [T][top_k] fp32 out.
+ * A token with a NaN score (NaN in x, w_router or bias) gets index -1 (which
+ * moe_union rejects) and weight 0 in every slot, and MOE_EDEVICE_INDEX is
+ * recorded in the workspace status word.
  * T = 0 is a no-op.  Errors: MOE_EINVAL, MOE_EWORKSPACE, MOE_ECUDA.
  */
 int moe_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
@@ -153,7 +156,8 @@ int moe_route(const uint16_t* x, int T, int H, const float* w_router, const floa
  *  - Every call in the process shares the one array per device and leaves its
  *    logits there.  Calls whose kernels may overlap on the same device (on
  *    different streams, or from different threads) race on it: order them.
- *  - Unlike moe_route it records no device-side status word.
+ *  - Unlike moe_route it records no device-side status word; a token with a
+ *    NaN score still gets index -1 and weight 0 in every slot.
  */
 int moe_route_noalloc(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
                       const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w,

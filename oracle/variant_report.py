@@ -37,18 +37,13 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 from oracle import oracle as O  # noqa: E402
+from oracle.synth_inputs import oracle_experts  # noqa: E402
 
 VARIANTS = ("", "silu32", "muladd", "silu32_muladd")
 
 
 def _experts(sh, ids, shared=False):
-    ex = O.Experts(sh.qtype, sh.H, sh.I, 1 if shared else sh.E)
-    for e in ids:
-        sid = synth.SHARED if shared else int(e)
-        mats = [synth.expert_matrix(sh, 0, sid, m) for m in (synth.GATE, synth.UP, synth.DOWN)]
-        ex.set(0 if shared else int(e), mats[0][0], mats[0][1], mats[1][0], mats[1][1], mats[2][0],
-               mats[2][1])
-    return ex
+    return oracle_experts(sh, ids, shared=shared)
 
 
 def layer_outputs(sh, batches, variant: str = ""):

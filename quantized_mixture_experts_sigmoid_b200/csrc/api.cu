@@ -6,10 +6,21 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
 using namespace moe;
+
+namespace {
+// An NVTX range named after the entry point, open for the call's duration
+// (visible in profilers; without one attached it costs a few nanoseconds).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
 
 namespace moe {
 
@@ -33,6 +44,16 @@ std::atomic<long long> g_launches{0};
 }
 
 void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int check_cfg(const moe_router_cfg* c) {
+    if (!c) return MOE_EINVAL;
+    const int E = c->n_expert, G = c->n_group;
+    if (E <= 0 || E > 1024 || G <= 0 || G > 32 || E % G != 0 || E / G < 2) return MOE_EINVAL;
+    if (c->topk_group <= 0 || c->topk_group > G) return MOE_EINVAL;
+    if (c->top_k <= 0 || c->top_k > 32 || c->top_k > c->topk_group * (E / G)) return MOE_EINVAL;
+    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_EINVAL;
+    return MOE_OK;
+}
 
 }  // namespace moe
 
@@ -61,16 +82,6 @@ Profiler g_prof;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
-
-int check_cfg(const moe_router_cfg* c) {
-    if (!c) return MOE_EINVAL;
-    const int E = c->n_expert, G = c->n_group;
-    if (E <= 0 || E > 1024 || G <= 0 || G > 32 || E % G != 0 || E / G < 2) return MOE_EINVAL;
-    if (c->topk_group <= 0 || c->topk_group > G) return MOE_EINVAL;
-    if (c->top_k <= 0 || c->top_k > 32 || c->top_k > c->topk_group * (E / G)) return MOE_EINVAL;
-    if (!(c->routed_scaling_factor == c->routed_scaling_factor)) return MOE_EINVAL;
-    return MOE_OK;
-}
 
 int check_experts(const moe_experts* ex) {
     if (!ex) return MOE_EINVAL;
@@ -267,6 +278,7 @@ size_t moe_route_workspace_bytes(int T, const moe_router_cfg* cfg) {
 int moe_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
               const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w, void* ws,
               size_t ws_bytes, moe_stream_t stream) {
+    NvtxRange nvtx("moe_route");
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (T < 0 || H <= 0 || H % 32) return MOE_EINVAL;
@@ -286,6 +298,7 @@ int moe_route(const uint16_t* x, int T, int H, const float* w_router, const floa
 int moe_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_unique, int32_t* uniq,
               int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot, int32_t* counts,
               int32_t* status, moe_stream_t stream) {
+    NvtxRange nvtx("moe_union");
     if (T < 0 || top_k <= 0 || top_k > 32 || E <= 0 || E > 1024) return MOE_EINVAL;
     if (!n_unique || !uniq || !offsets) return MOE_EINVAL;
     if (T > 0 && (!topk_idx || !pair_tok || !pair_slot)) return MOE_EINVAL;
@@ -296,6 +309,7 @@ int moe_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_uniqu
 
 int moe_quantize_q8_0(const void* v, int in_dtype, int rows, int n, int8_t* q, float* d,
                       moe_stream_t stream) {
+    NvtxRange nvtx("moe_quantize_q8_0");
     if (rows < 0 || n <= 0 || n % 32) return MOE_EINVAL;
     if (in_dtype != MOE_OUT_BF16 && in_dtype != MOE_OUT_F32) return MOE_EINVAL;
     if (rows == 0) return MOE_OK;
@@ -313,6 +327,7 @@ int moe_expert_ffn_q(const moe_experts* ex, const uint16_t* x, int T, int top_k,
                      const int32_t* n_unique, const int32_t* uniq, const int32_t* offsets,
                      const int32_t* pair_tok, const int32_t* pair_slot, float* y_pairs, void* ws,
                      size_t ws_bytes, moe_stream_t stream) {
+    NvtxRange nvtx("moe_expert_ffn_q");
     int rc = check_experts(ex);
     if (rc) return rc;
     if (T < 0 || top_k <= 0 || top_k > 32) return MOE_EINVAL;
@@ -339,6 +354,7 @@ int moe_expert_ffn_q(const moe_experts* ex, const uint16_t* x, int T, int top_k,
 
 int moe_combine(const float* y_pairs, const float* topk_w, const float* shared_y, int T, int top_k,
                 int H, void* out, int out_dtype, moe_stream_t stream) {
+    NvtxRange nvtx("moe_combine");
     if (T < 0 || top_k <= 0 || top_k > 32 || H <= 0 || H % 4) return MOE_EINVAL;
     if (out_dtype != MOE_OUT_BF16 && out_dtype != MOE_OUT_F32) return MOE_EINVAL;
     if (T == 0) return MOE_OK;
@@ -360,6 +376,7 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
                       const moe_router_cfg* cfg, const moe_experts* routed,
                       const moe_experts* shared, void* out, int out_dtype, int32_t* topk_idx_out,
                       float* topk_w_out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    NvtxRange nvtx("moe_layer_forward");
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if ((rc = check_experts(routed))) return rc;
@@ -506,6 +523,7 @@ int moe_profile_read(double* total_ms, int* launches) {
 long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream) {
+    NvtxRange nvtx("moe_workspace_status");
     if (!ws || !status) return MOE_EINVAL;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     int32_t h = 0;

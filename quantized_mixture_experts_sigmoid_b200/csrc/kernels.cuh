@@ -13,6 +13,10 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes);
 // Adds n to the process-wide count of kernels this library launched.
 void count_launch(int n = 1);
 
+// MOE_OK or MOE_EINVAL: the router configuration limits of moe.h (every
+// entry point that takes a moe_router_cfg checks it with this function).
+int check_cfg(const moe_router_cfg* c);
+
 // Returns e after counting one launch when it succeeded.
 inline cudaError_t counted(cudaError_t e) {
     if (e == cudaSuccess) count_launch(1);

@@ -48,12 +48,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 extern "C" int moe_route_noalloc(const uint16_t* x, int T, int H, const float* w_router,
                                  const float* bias, const moe_router_cfg* cfg, int32_t* topk_idx,
                                  float* topk_w, moe_stream_t stream) {
-    if (!cfg) return MOE_EINVAL;
-    const int E = cfg->n_expert, G = cfg->n_group;
-    if (E <= 0 || E > 1024 || G <= 0 || G > 32 || E % G != 0 || E / G < 2) return MOE_EINVAL;
-    if (cfg->topk_group <= 0 || cfg->topk_group > G) return MOE_EINVAL;
-    if (cfg->top_k <= 0 || cfg->top_k > 32 || cfg->top_k > cfg->topk_group * (E / G)) return MOE_EINVAL;
-    if (!(cfg->routed_scaling_factor == cfg->routed_scaling_factor)) return MOE_EINVAL;
+    const int rc = moe::check_cfg(cfg);  // the same limits as moe_route
+    if (rc) return rc;
+    const int E = cfg->n_expert;
     if (T < 0 || H <= 0 || H % 32) return MOE_EINVAL;
     if (T == 0) return MOE_OK;
     if (static_cast<long long>(T) * E > MOE_ROUTE_NOALLOC_MAX_LOGITS) return MOE_ETOO_LARGE;

@@ -22,13 +22,26 @@ __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __
                                                   float* s, float* b, int* chosen,
                                                   int32_t* idx, float* w, int32_t* status) {
     const int lane = threadIdx.x & 31;
+    bool nan = false;
     for (int e = lane; e < E; e += 32) {
         const double l = static_cast<double>(logit(e));
         const float sv = __double2float_rn(1.0 / (1.0 + exp(-l)));
         s[e] = sv;
         b[e] = __fadd_rn(sv, __ldg(bias + e));
+        nan |= b[e] != b[e];
     }
     __syncwarp();
+    if (__any_sync(0xffffffffu, nan)) {
+        // a NaN score leaves no expert choosable: every slot gets index -1
+        // (which moe_union rejects) and weight 0
+        record_status(status, MOE_EDEVICE_INDEX);
+        for (int k = lane; k < K; k += 32) {
+            idx[k] = -1;
+            w[k] = 0.0f;
+        }
+        __syncwarp();
+        return;
+    }
     const int gsz = E / G;
     float gs = -INFINITY;
     if (lane < G) {
@@ -50,9 +63,9 @@ __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __
         float v = ok ? gs : -INFINITY;
         int i = ok ? lane : 0x7fffffff;
         warp_argmax(v, i);
-        if (i >= G) {  // only reachable with NaN scores: keep indices in range, flag it
+        if (i >= G) {  // only reachable with NaN scores: no group is kept for this round
             record_status(status, MOE_EDEVICE_INDEX);
-            i = 0;
+            continue;
         }
         keep |= 1u << i;
     }
@@ -68,23 +81,26 @@ __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __
             }
         }
         warp_argmax(best, bi);
-        if (bi >= E) {  // only reachable with NaN scores
+        if (bi >= E) {  // only reachable with NaN scores: no expert for this slot
             record_status(status, MOE_EDEVICE_INDEX);
-            bi = 0;
+            bi = -1;
         }
         if (lane == 0) {
             chosen[k] = bi;
-            b[bi] = -INFINITY;
+            if (bi >= 0) b[bi] = -INFINITY;
         }
         __syncwarp();
     }
     if (lane == 0) {
+        // a slot left without an expert (NaN scores) gets index -1, which
+        // moe_union rejects, and weight 0
         float den = 0.0f;
-        for (int k = 0; k < K; ++k) den = __fadd_rn(den, s[chosen[k]]);
+        for (int k = 0; k < K; ++k)
+            if (chosen[k] >= 0) den = __fadd_rn(den, s[chosen[k]]);
         for (int k = 0; k < K; ++k) {
             const int e = chosen[k];
             idx[k] = e;
-            w[k] = __fmul_rn(__fdiv_rn(s[e], den), rsf);
+            w[k] = e >= 0 ? __fmul_rn(__fdiv_rn(s[e], den), rsf) : 0.0f;
         }
     }
     __syncwarp();

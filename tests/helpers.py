@@ -7,20 +7,8 @@ from __future__ import annotations
 import numpy as np
 
 import synth
-from oracle import oracle as O
-
-
-def oracle_experts(sh: synth.LayerShape, experts, layer: int = 0, shared: bool = False):
-    """Oracle expert set holding only the listed experts (regenerated from the seed)."""
-    n = 1 if shared else sh.E
-    ex = O.Experts(sh.qtype, sh.H, sh.I, n)
-    for e in experts:
-        sid = synth.SHARED if shared else int(e)
-        g, sg = synth.expert_matrix(sh, layer, sid, synth.GATE)
-        u, su = synth.expert_matrix(sh, layer, sid, synth.UP)
-        d, sd = synth.expert_matrix(sh, layer, sid, synth.DOWN)
-        ex.set(0 if shared else int(e), g, sg, u, su, d, sd)
-    return ex
+from oracle import oracle as O  # noqa: F401
+from oracle.synth_inputs import oracle_experts  # noqa: F401
 
 
 def layer_inputs(sh: synth.LayerShape, layer: int = 0, tokens=None):

@@ -356,3 +356,33 @@ def test_layer_forward_repeated_calls_reuse_workspace():
     for o in outs[1:]:
         assert np.array_equal(o.cpu().numpy().view(np.uint32), first.view(np.uint32))
     check_layer(sh, dev, x, W, b)
+
+
+def test_route_nan_token_gets_no_expert():
+    # a token whose scores are NaN cannot be routed: every slot gets index -1
+    # and weight 0 (moe_union rejects -1), the workspace router records the code,
+    # and the other tokens of the batch are routed as usual
+    sh = SHAPES["ragged"]
+    dev = dict(W=torch.from_numpy(synth.router_weight(sh)).cuda(),
+               bias=torch.from_numpy(synth.router_bias(sh)).cuda(),
+               cfg=moe.RouterCfg(sh.E, sh.n_group, sh.topk_group, sh.top_k, sh.rsf))
+    x, W, b = layer_inputs(sh)
+    x = x.copy()
+    x[3, 7] = 0x7FC0  # bf16 quiet NaN
+    idx_o, w_o, _, _ = O.route(np.delete(x, 3, axis=0), W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+    for noalloc in (False, True):
+        idx = torch.empty(sh.T, sh.top_k, dtype=torch.int32, device="cuda")
+        w = torch.empty(sh.T, sh.top_k, dtype=torch.float32, device="cuda")
+        xd = to_dev_bf16(x)
+        if noalloc:
+            moe.moe_route_noalloc(xd, dev["W"], dev["bias"], dev["cfg"], idx, w)
+        else:
+            ws = moe.workspace(moe.moe_route_workspace_bytes(sh.T, dev["cfg"]))
+            moe.moe_route(xd, dev["W"], dev["bias"], dev["cfg"], idx, w, ws)
+            assert moe.moe_workspace_status(ws) == moe.MOE_EDEVICE_INDEX
+        ig, wg = idx.cpu().numpy(), w.cpu().numpy()
+        assert np.all(ig[3] == -1) and np.all(wg[3] == 0.0)
+        assert np.array_equal(np.delete(ig, 3, axis=0), idx_o)
+        assert np.array_equal(np.delete(wg, 3, axis=0).view(np.uint32), w_o.view(np.uint32))
+        g = gpu_union(ig, sh.E)
+        assert g["status"] == moe.MOE_EDEVICE_INDEX
