@@ -13,27 +13,27 @@
 //    with bulk copies (cp.async.bulk, non-multicast TMA) completing on
 //    mbarriers;
 //  * warps 0-15, the consumers, take one ring stage at a time and form the
-//    integer dot products with dp4a;
+//    integer dot products with dp4a; once their router rows are done they
+//    also route the batch (every CTA computes the same routing from the
+//    published router scores, one expert per thread);
 //  * warps 16-17, the epilogue warps, each finish the tiles handed over
 //    through one task slot (SwiGLU and Q8_0 of h for up/gate tiles;
 //    completion counting and the combine for down tiles), so the consumers
 //    never wait on fences or atomics;
-//  * warp 19, the helper, first routes the batch (every CTA computes the same
-//    routing from the published router scores, in registers), then copies
-//    each down tile's activation records once the expert's h is complete, so
-//    the producer never waits on another CTA.
+//  * warp 19, the helper, copies each down tile's activation records once
+//    the expert's h is complete, so the producer never waits on another CTA.
 //
 // Work is one global ticket sequence claimed by the producers:
 //      router rows | shared up/gate tiles | then, per distinct routed expert
-//      u: its up/gate tiles, followed by the down tiles of expert u - 3; the
+//      u: its up/gate tiles, followed by the down tiles of expert u - 8; the
 //      last routed experts' down tiles at the end, the shared expert's down
 //      tiles before the very last expert's,
 // so every dependency points to an earlier ticket, far enough back that it is
 // usually complete when claimed.  The consumers that finish a router row
 // publish its scores (sigmoid of the fp32-rounded logit) in 64-bit slots
-// tagged with the launch number; the helper warps poll those slots, so the
-// data and its readiness arrive in one load.  A producer claims routed tiles
-// once its helper warp has routed.  An up/gate tile is 32 rows of h for one
+// tagged with the launch number; every CTA's consumers poll those slots, so
+// the data and its readiness arrive in one load.  A producer claims routed
+// tiles once its CTA's consumers have routed.  An up/gate tile is 32 rows of h for one
 // expert; its epilogue writes Q8_0(h) as a pre-permuted activation record.  A
 // down tile's weight stages stream at once; its records follow when the
 // expert's h tiles are all done.  The CTA that completes a row block of the
@@ -93,7 +93,7 @@ static_assert(kDownStagesPerTile == kGroups && (2 * (kUgTileRows / kStageRows)) 
 constexpr int kDownLag = 8;          // routed experts between an expert's up/gate and down tiles
 constexpr int kMaxExpertsPerLane = 8; // warp routing: E <= 32 * 8
 
-enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3 };
+enum : int { D_EXIT = 0, D_ROUTER = 1, D_UG = 2, D_DOWN = 3, D_MARK = 4 };  // D_MARK: route now
 constexpr int kMaxPairs = kMaxT * 32;
 
 struct Desc {
@@ -133,10 +133,30 @@ struct Task {
     int pair[kMaxT];
 };
 
+using u64 = unsigned long long;
+
+// Routing scratch, one half per token routed at the same time.  It lives in
+// the x cache, which is free once Q8_0(x) is built.
+struct alignas(16) RouteHalf {
+    u64 cand[32 * kMaxExpertsPerLane];   // (key, complement of the index) of every expert
+    float sc[32 * kMaxExpertsPerLane];   // scores s (unbiased)
+    uint32_t part[kMaxExpertsPerLane][2];  // per warp of 32 experts: largest, second largest key
+    int slot[kMaxExpertsPerLane];        // the expert of each slot
+    uint32_t kept;                       // kept groups
+    int nan;
+};
+// the rank scan reads cand as 16-byte pairs, in both halves
+static_assert(sizeof(RouteHalf) % 16 == 0, "each half's cand array must stay 16-byte aligned");
+struct RouteScratch {
+    RouteHalf h[2];
+    int pe[kMaxPairs];                   // expert of pair t K + k
+    int bad[kMaxT];                      // token t had a NaN score
+};
+
 struct Smem {
     uint8_t* ring;
     uint8_t* act;
-    uint16_t* xs;    // bf16 x; reused as routing scratch once the router rows are done
+    uint16_t* xs;    // bf16 x; the routing scratch (RouteScratch) once Q8_0(x) is built
     uint4* q0;
     uint4* q1;
     float* qd;
@@ -181,7 +201,7 @@ __host__ __device__ inline Layout layout_of(const FusedParams& p) {
     size_t o = 0;
     L.ring = o; o += a16(slot * p.nstage);
     L.act = o; o += a16(static_cast<size_t>(p.act_bytes) * kActSlots);
-    L.xs = o; o += a16(static_cast<size_t>(p.T) * p.H * 2);
+    L.xs = o; o += a16(std::max(static_cast<size_t>(p.T) * p.H * 2, sizeof(RouteScratch)));
     L.qx = o; o += a16(static_cast<size_t>(p.T) * nbH * 40);
     L.bias = o; o += a16(sizeof(float) * p.E);
     L.desc = o; o += a16(sizeof(Desc) * p.nstage);
@@ -356,6 +376,21 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         return true;
     };
 
+    // One marker stage per consumer group, ahead of the first stage that is
+    // not a router row: the consumers route when they reach it, so they never
+    // wait for a stage that itself waits for the routing.
+    bool marked = false;
+    auto mark = [&]() -> bool {
+        marked = true;
+        for (int g = 0; g < kGroups; ++g) {
+            if (!acquire_stage()) return false;
+            s.desc[stage].type = D_MARK;
+            mbar_arrive(&s.full[stage]);
+            advance();
+        }
+        return true;
+    };
+
     // The first ticket of CTA b is b: no round trip before the first copy,
     // and none of the workspace is touched, so it streams while the previous
     // grid in the stream finishes.  Later tickets come from the shared
@@ -377,6 +412,10 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
             d.nrows = min(p.rps, p.E - d.e);
             ok = issue(d, p.w_router + static_cast<size_t>(d.e) * p.H, 4u * p.H * d.nrows, nullptr, 0);
             continue;
+        }
+        if (!marked && !mark()) {
+            ok = false;
+            break;
         }
         int t = cur - nrt;
         int kind, u, j;  // kind: 0 up/gate, 1 down; u = -1 shared
@@ -474,6 +513,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         }
     }
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
+    if (!marked) mark();  // the consumers route before they look for the end
     // tell the helper warp and the consumers to stop
     if (mbar_wait(&s.areq_free[aslot], aphase ^ 1u, kProducerWait)) {
         s.areq[aslot].exit = 1;
@@ -658,13 +698,6 @@ __device__ void consume_router(const FusedParams& p, const Smem& s, int e0, int 
     group_sync(g);  // the reduction buffer is reused by this group's next router stage
 }
 
-// Selection and union for the whole batch, computed by all consumer threads
-// of every CTA into shared memory once every logit has been counted.
-// noaux_tc (DeepSeek-V3 routing, as [HN] "구현된 주요 기능" names it):
-// s = sigmoid(logit), b = s + bias; group score = sum of the two largest b;
-// keep topk_group groups; keep the top_k experts of kept groups by b; ties to
-// the lower index.  A kept group / expert finds its rank by counting the
-// candidates that order before it (vectorised scans over shared memory).
 // Order-preserving map of fp32 values to unsigned keys (+0 and -0 equal; the
 // key 0 is below every value and marks an excluded expert).
 __device__ __forceinline__ uint32_t order_key(float v) {
@@ -676,195 +709,182 @@ __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Compare-exchange of two (key, expert, score) candidates so that the first
-// is the better one: larger key, then lower expert index.
-__device__ __forceinline__ void cand_order(uint32_t& ka, int& ea, float& sa, uint32_t& kb, int& eb, float& sb) {
-    const bool swap = kb > ka || (kb == ka && eb < ea);
-    const uint32_t k = swap ? kb : ka;
-    const int e = swap ? eb : ea;
-    const float v = swap ? sb : sa;
-    kb = swap ? ka : kb;
-    eb = swap ? ea : eb;
-    sb = swap ? sa : sb;
-    ka = k;
-    ea = e;
-    sa = v;
+__device__ __forceinline__ uint32_t max_u32(uint32_t a, uint32_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint32_t min_u32(uint32_t a, uint32_t b) { return a < b ? a : b; }
+
+// Merges the (largest, second largest) pair (b1, b2) into (a1, a2); a maximum
+// held twice counts twice.
+__device__ __forceinline__ void top2_merge(uint32_t& a1, uint32_t& a2, uint32_t b1, uint32_t b2) {
+    a2 = max_u32(min_u32(a1, b1), max_u32(a2, b2));
+    a1 = max_u32(a1, b1);
 }
 
-// noaux_tc routing and the batch union of the whole batch by one warp, with
-// each lane holding experts lane + 32 j of a token in registers (E <= 256,
-// groups of a multiple of 32 experts, T K <= 32).  Per token: group score =
-// sum of the two largest biased scores (warp max reductions); the TG best
-// groups kept (ties to the lower group); then each lane sorts its kept
-// candidates (larger biased score, then lower index) and K rounds of a warp
-// arg-max over the lanes' best remaining candidate give the slots in order.
-// Gate weights use the unbiased scores, their sum taken in slot order.  The
-// union lists the pairs by (expert, token).  Runs on the helper warp, in
-// parallel with the consumers, which never wait for it; the producer waits on
-// route_bar.
-__device__ __forceinline__ void route_warp(const FusedParams& p, const Smem& s) {
-    constexpr int NJ = kMaxExpertsPerLane;
-    const int lane = threadIdx.x & 31;
-    const int T = p.T, K = p.K, E = p.E, G = p.G, TG = p.TG, NE = E >> 5, m = NE / G;
+// noaux_tc routing (DeepSeek-V3 routing, as [HN] "구현된 주요 기능" names it)
+// and the batch union, by all consumer threads: each half of them (256
+// threads, one expert each) routes one token, two tokens at a time.
+//   b = s + bias (fp32); group score = sum of the group's two largest b (a
+//   maximum held twice counts twice); the TG best groups kept, ties to the
+//   lower group; the top K experts of the kept groups by b fill the slots in
+//   order, ties to the lower index; gate weight of slot k = s_k / (s_0 + ...
+//   + s_{K-1}) * rsf with the sum taken in slot order.
+// The routed weight stream cannot start before routing ends, so the work is
+// spread for a short chain per thread: each warp (32 experts) reduces its
+// (largest, second) pair by a butterfly, one warp sums and ranks the groups,
+// and every candidate of a kept group counts the kept candidates that order
+// before it (key, then lower index: one compare of 64-bit words).  The union
+// lists the pairs by (expert, token).  Thread 0 then releases the producer
+// through route_bar.
+// A token with a NaN score is still given K valid experts internally (the
+// ticket sequence needs them) but reports index -1 and weight 0 to the caller
+// and records MOE_EDEVICE_INDEX; its output row is unspecified.
+__device__ void route_block(const FusedParams& p, const Smem& s) {
+    const int tid = threadIdx.x, half = tid >> 8, e = tid & 255, lane = tid & 31, hw = e >> 5;
+    const int T = p.T, K = p.K, E = p.E, G = p.G, TG = p.TG, gsz = E / G, wpg = gsz >> 5;
+    RouteScratch* rs = reinterpret_cast<RouteScratch*>(s.xs);
+    RouteHalf& h = rs->h[half];
     const uint32_t tag = *s.tag;
-    float bias_r[NJ];
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) bias_r[j] = j < NE ? __ldg(p.bias + lane + 32 * j) : 0.0f;
     bool ok = true;
-    int pe = 0;  // lane t K + k: expert of token t, slot k
-    float pw = 0.0f;
-    for (int t = 0; t < T; ++t) {
-        // this token's scores, as soon as every slot carries this launch's tag
-        float sc[NJ];
-        uint32_t pend = (1u << NE) - 1u;
+    for (int t0 = 0; t0 < T; t0 += 2) {
+        const int t = t0 + half;
+        const bool tok = t < T, live = tok && e < E;
+        // this token's score of expert e, once it carries this launch's tag
+        float sc = 0.0f;
+        if (live) {
+            for (long it = 0;; ++it) {
+                const u64 v = ld_relaxed_gpu_u64(p.scores + static_cast<size_t>(t) * E + e);
+                if (static_cast<uint32_t>(v >> 32) == tag) {
+                    sc = __uint_as_float(static_cast<uint32_t>(v));
+                    break;
+                }
+                if (it >= kConsumerWait) {
+                    ok = false;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        const float b = live ? __fadd_rn(sc, s.bias[e]) : 0.0f;
+        const uint32_t key = live ? order_key(b) : 0u;
+        h.sc[e] = sc;
+        h.cand[e] = (static_cast<u64>(key) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(e));
+        uint32_t t1 = key, t2 = 0u;
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) sc[j] = 0.0f;
-        for (long it = 0; ok; ++it) {
-            // all loads first (their predicates must not depend on earlier
-            // loads' results, or they would be issued one after another)
-            unsigned long long v[NJ];
-            const uint32_t want = pend;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j)
-                v[j] = ((want >> j) & 1u) ? ld_relaxed_gpu_u64(p.scores + t * E + lane + 32 * j) : 0ull;
-#pragma unroll
-            for (int j = 0; j < NJ; ++j) {
-                if (((want >> j) & 1u) && static_cast<uint32_t>(v[j] >> 32) == tag) {
-                    sc[j] = __uint_as_float(static_cast<uint32_t>(v[j]));
-                    pend &= ~(1u << j);
+        for (int o = 16; o > 0; o >>= 1)
+            top2_merge(t1, t2, __shfl_xor_sync(0xffffffffu, t1, o), __shfl_xor_sync(0xffffffffu, t2, o));
+        const bool nan = __any_sync(0xffffffffu, live && b != b);
+        if (lane == 0) {
+            h.part[hw][0] = t1;
+            h.part[hw][1] = t2;
+            if (hw == 0) h.nan = 0;
+        }
+        consumers_sync();
+        if (nan && lane == 0) h.nan = 1;
+        // group scores and the kept groups, by the first warp of the half
+        if (hw == 0 && tok) {
+            float gs = 0.0f;
+            if (lane < G) {
+                uint32_t a1 = 0u, a2 = 0u;
+                for (int w = lane * wpg; w < lane * wpg + wpg; ++w) top2_merge(a1, a2, h.part[w][0], h.part[w][1]);
+                gs = __fadd_rn(key_value(a1), key_value(a2));
+            }
+            int r = 0;
+            for (int g = 0; g < G; ++g) {
+                const float o = __shfl_sync(0xffffffffu, gs, g);
+                r += (o > gs) || (o == gs && g < lane);
+            }
+            const uint32_t kept = __ballot_sync(0xffffffffu, lane < G && r < TG);
+            if (lane == 0) h.kept = kept;
+        }
+        consumers_sync();
+        // rank of each kept candidate among the kept candidates
+        const uint32_t kept = h.kept;
+        if (live && ((kept >> (e / gsz)) & 1u)) {
+            const u64 mine = h.cand[e];
+            int rank = 0;
+            for (uint32_t km = kept; km; km &= km - 1) {
+                const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(h.cand + (__ffs(km) - 1) * gsz);
+                for (int i = 0; i < gsz / 2; ++i) {
+                    const ulonglong2 v = c2[i];
+                    rank += (v.x > mine) + (v.y > mine);
                 }
             }
-            if (__all_sync(0xffffffffu, pend == 0)) break;
-            if (it >= kProducerWait) ok = false;
-            __nanosleep(32);
+            if (rank < K) h.slot[rank] = e;
         }
-        uint32_t key[NJ];
+        consumers_sync();
+        // slot k of token t: expert and gate weight
+        if (tok && e < K) {
+            int ex[kMaxExpertsPerLane];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) key[j] = j < NE ? order_key(__fadd_rn(sc[j], bias_r[j])) : 0u;
-        // group g = rows j in [g m, g m + m): the two largest keys of the
-        // group (equal maxima in two lanes count twice), summed as values
-        float gsum[NJ];
+            for (int k = 0; k < kMaxExpertsPerLane; ++k) ex[k] = k < K ? h.slot[k] : 0;
+            float den = 0.0f, mys = 0.0f;
 #pragma unroll
-        for (int g = 0; g < NJ; ++g) {
-            uint32_t k1 = 0, k2 = 0;
-            if (m == 1) {  // one row per group (32 experts)
-                k1 = g < G ? key[g] : 0u;
-            } else {
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    if (g < G && j >= g * m && j < g * m + m) {
-                        k2 = max(k2, min(k1, key[j]));
-                        k1 = max(k1, key[j]);
-                    }
+            for (int k = 0; k < kMaxExpertsPerLane; ++k) {
+                if (k < K) {
+                    const float sk = h.sc[ex[k]];
+                    den = __fadd_rn(den, sk);
+                    if (k == e) mys = sk;
                 }
             }
-            const uint32_t m1 = __reduce_max_sync(0xffffffffu, k1);
-            const uint32_t at = __ballot_sync(0xffffffffu, k1 == m1);
-            const uint32_t r2 = __reduce_max_sync(0xffffffffu, (k1 == m1 && (at & ((1u << lane) - 1u)) == 0) ? k2 : k1);
-            gsum[g] = __fadd_rn(key_value(m1), key_value(r2));
+            rs->pe[t * K + e] = h.slot[e];
+            s.rt_w[t * K + e] = __fmul_rn(__fdiv_rn(mys, den), p.rsf);
         }
-        // kept groups: each lane ranks group `lane` against the others
-        float mine = 0.0f;
-#pragma unroll
-        for (int g = 0; g < NJ; ++g)
-            if (g == lane) mine = gsum[g];
-        int r = 0;
-#pragma unroll
-        for (int g = 0; g < NJ; ++g) r += g < G && ((gsum[g] > mine) || (gsum[g] == mine && g < lane));
-        const uint32_t kept = __ballot_sync(0xffffffffu, lane < G && r < TG);
-        uint32_t kept_rows = 0;  // rows j of the kept groups
-#pragma unroll
-        for (int g = 0; g < NJ; ++g)
-            if (g < G && ((kept >> g) & 1u)) kept_rows |= ((1u << m) - 1u) << (g * m);
-        // this lane's candidates of the kept groups, sorted (best first) by an
-        // optimal 19-comparator network for 8 inputs
-        uint32_t ck[NJ];
-        int ce[NJ];
-        float cs[NJ];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            ck[j] = ((kept_rows >> j) & 1u) ? key[j] : 0u;
-            ce[j] = lane + 32 * j;
-            cs[j] = sc[j];
-        }
-        static_assert(NJ == 8, "sorting network is for 8 candidates");
-        constexpr int kNet[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6}, {5, 7}, {1, 2}, {5, 6},
-                                     {0, 4}, {3, 7}, {1, 5}, {2, 6}, {1, 4}, {3, 6}, {2, 4}, {3, 5}, {3, 4}};
-#pragma unroll
-        for (int c = 0; c < 19; ++c) {
-            const int a = kNet[c][0], b = kNet[c][1];
-            cand_order(ck[a], ce[a], cs[a], ck[b], ce[b], cs[b]);
-        }
-        // K rounds: the warp's best head wins; its lane pops it
-        int my_e = -1;
-        float my_s = 0.0f, den = 0.0f;
-        for (int k = 0; k < K; ++k) {
-            const uint32_t mx = __reduce_max_sync(0xffffffffu, ck[0]);
-            const uint32_t win = __reduce_min_sync(0xffffffffu, (ck[0] == mx && mx != 0u) ? static_cast<uint32_t>(ce[0]) : 0xffffffffu);
-            const bool mine_w = static_cast<uint32_t>(ce[0]) == win;
-            const float sw = __shfl_sync(0xffffffffu, cs[0], win & 31u);
-            den = __fadd_rn(den, sw);  // slot order
-            if (lane == k) {
-                my_e = static_cast<int>(win);
-                my_s = sw;
-            }
-            if (mine_w) {
-#pragma unroll
-                for (int j = 0; j < NJ - 1; ++j) {
-                    ck[j] = ck[j + 1];
-                    ce[j] = ce[j + 1];
-                    cs[j] = cs[j + 1];
-                }
-                ck[NJ - 1] = 0u;
-            }
-        }
-        if (lane < K && (my_e < 0 || my_e >= E)) {  // only reachable with NaN scores
-            record_status(p.status, MOE_EDEVICE_INDEX);
-            my_e = 0;
-        }
-        const float my_w = __fmul_rn(__fdiv_rn(my_s, den), p.rsf);
-        // move token t's K results to lanes t K .. t K + K - 1
-        const int src = lane - t * K;
-        const int e_t = __shfl_sync(0xffffffffu, my_e, src & 31);
-        const float w_t = __shfl_sync(0xffffffffu, my_w, src & 31);
-        if (src >= 0 && src < K) {
-            pe = e_t;
-            pw = w_t;
-        }
+        if (tok && e == 0) rs->bad[t] = h.nan;
+        consumers_sync();
     }
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
-    // batch union: pair position = number of pairs with a smaller (expert, token)
+    if (tid >= 32) return;
+    // the batch union, by warp 0
+    const unsigned all = 0xffffffffu;
+    uint32_t bad_tokens = 0;  // bit t: token t had a NaN score
+    for (int t = 0; t < T; ++t) bad_tokens |= rs->bad[t] ? 1u << t : 0u;
+    if (bad_tokens && lane == 0) record_status(p.status, MOE_EDEVICE_INDEX);
     const int n = T * K;  // <= 32
     const bool act = lane < n;
-    const int key = act ? (pe << 5) | lane : 0x7fffffff;
-    const uint32_t same = T > 1 ? __match_any_sync(0xffffffffu, act ? pe : -1 - lane) : (1u << lane);
-    const bool first = act && (__ffs(same) - 1 == lane);
-    const uint32_t firsts = __ballot_sync(0xffffffffu, first);
-    int pos = 0, urank = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const int kj = __shfl_sync(0xffffffffu, key, j);
-        if (j < n) {
+    const int pe = act ? rs->pe[lane] : 0;
+    const float pw = act ? s.rt_w[lane] : 0.0f;
+    if (T == 1) {
+        // one token: K distinct experts; a pair's position is its expert's rank
+        int pos = 0;
+        for (int k = 0; k < K; ++k) pos += rs->pe[k] < pe;
+        if (act) {
+            s.rt_ptok[pos] = 0;
+            s.rt_pair_of[lane] = pos;
+            s.rt_uniq[pos] = pe;
+            s.rt_off[pos] = pos;
+        }
+        if (lane == 0) {
+            *s.rt_U = K;
+            s.rt_off[K] = K;
+        }
+    } else {
+        // pair position = number of pairs with a smaller (expert, token)
+        const int key = act ? (pe << 5) | lane : 0x7fffffff;
+        const uint32_t same = __match_any_sync(all, act ? pe : -1 - lane);
+        const bool first = act && (__ffs(same) - 1 == lane);
+        const uint32_t firsts = __ballot_sync(all, first);
+        int pos = 0, urank = 0;
+        for (int j = 0; j < n; ++j) {
+            const int kj = __shfl_sync(all, key, j);
             pos += kj < key;
             urank += ((firsts >> j) & 1u) && (kj >> 5) < pe;
         }
-    }
-    if (act) {
-        s.rt_ptok[pos] = lane / K;
-        s.rt_pair_of[lane] = pos;
-        s.rt_w[lane] = pw;
-        if (first) {
-            s.rt_uniq[urank] = pe;
-            s.rt_off[urank] = pos;
+        if (act) {
+            s.rt_ptok[pos] = lane / K;
+            s.rt_pair_of[lane] = pos;
+            if (first) {
+                s.rt_uniq[urank] = pe;
+                s.rt_off[urank] = pos;
+            }
         }
-        if (blockIdx.x == 0) {  // the routing the caller can see, written once
-            p.idx[lane] = pe;
-            p.w[lane] = pw;
+        if (lane == 0) {
+            *s.rt_U = __popc(firsts);
+            s.rt_off[__popc(firsts)] = n;
         }
     }
-    if (lane == 0) {
-        *s.rt_U = __popc(firsts);
-        s.rt_off[__popc(firsts)] = n;
+    if (act && blockIdx.x == 0) {  // the routing the caller can see, written once
+        const bool bad = (bad_tokens >> (lane / K)) & 1u;
+        p.idx[lane] = bad ? -1 : pe;
+        p.w[lane] = bad ? 0.0f : pw;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(s.route_bar);
@@ -1093,15 +1113,19 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
         tb ^= 1;
     };
     int type = next_type();
-    // phase A: router rows (the helper warp routes meanwhile), then Q8_0 of x
+    // phase A: router rows up to the route marker, Q8_0 of x, then the routing
     while (type == D_ROUTER) {
         const int e0 = s.desc[stage].e, nrows = s.desc[stage].nrows;
         consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes, g);
         release();
         type = next_type();
     }
+    const bool marker = type == D_MARK;
+    if (marker) release();
     quantize_x<QT>(p, s);
     consumers_sync();
+    route_block(p, s);  // the x cache holds the routing scratch from here on
+    if (marker) type = next_type();
     // phases B and C: runs of up/gate tiles and of down tiles.  A tile's
     // stages alternate between the groups, so every warp sees every tile:
     // its first stage of a tile (sit < kGroups) claims the task slot or the
@@ -1200,12 +1224,11 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
 }
 
 // ------------------------------------------------------------------ helper warp
-// Routes the batch (all lanes), then lane 0 serves the producer's down-tile
-// requests in order: waits until the slot's previous records are consumed and
-// the expert's h tiles are all complete, then bulk-copies the records.
+// Lane 0 serves the producer's down-tile requests in order: waits until the
+// slot's previous records are consumed and the expert's h tiles are all
+// complete, then bulk-copies the records.
 template <int QT>
 __device__ __forceinline__ void helper_warp(const FusedParams& p, const Smem& s) {
-    route_warp(p, s);
     if ((threadIdx.x & 31) != 0) return;
     long n_act = 0;
     int slot = 0;
@@ -1385,7 +1408,8 @@ const void* fused_kernel(int nt) {
 bool fused_geometry(FusedParams& p, int qtype) {
     // one warp routes the batch: experts lane + 32 j in registers (E <= 256),
     // groups of a multiple of 32 experts, the batch's T K pairs in one warp
-    if (p.T < 1 || p.T > kMaxT || p.K < 1 || p.K * p.T > 32 || p.T * p.E > kFusedMaxSlots) return false;
+    if (p.T < 1 || p.T > kMaxT || p.K < 1 || p.K > kMaxExpertsPerLane || p.K * p.T > 32 || p.T * p.E > kFusedMaxSlots)
+        return false;
     if (p.E % 32 || p.E > 32 * kMaxExpertsPerLane || p.G < 1 || p.E % p.G || (p.E / p.G) % 32) return false;
     if (p.TG < 1 || p.TG > p.G || p.TG * (p.E / p.G) < p.K) return false;
     const size_t rb_ug = static_cast<size_t>(p.H) * qtype / 8, rb_d = static_cast<size_t>(p.I) * qtype / 8;
