@@ -73,7 +73,8 @@ constexpr int kUgTileRows = 32;      // one Q8_0 block of h
 constexpr int kDownStagesPerTile = 2;  // one per consumer group
 constexpr int kMaxRouterRows = 4;    // router rows per stage
 constexpr int kMaxDownRowsPerWarp = 8;
-constexpr int kActSlots = 2;
+constexpr int kActSlots = 2;         // activation-record slots of their own
+constexpr int kMaxActSlots = 6;      // with up to 4 more in the x cache, free once routed
 constexpr int kTaskSlots = kEpilogueWarps;
 constexpr int kScaleBytes = 256;     // room after each stage for its rows' fp32 scales
 // Copies a producer keeps in flight.  Enough to cover HBM latency at full
@@ -174,9 +175,9 @@ struct Smem {
     uint64_t* tfull;
     uint64_t* tfree;
     uint64_t* route_bar;  // helper warp -> producer: routing of the batch is ready
-    uint64_t* areq_full;  // [kActSlots] producer -> helper: request posted
-    uint64_t* areq_free;  // [kActSlots] helper -> producer: request taken
-    ActReq* areq;         // [kActSlots]
+    uint64_t* areq_full;  // [kMaxActSlots] producer -> helper: request posted
+    uint64_t* areq_free;  // [kMaxActSlots] helper -> producer: request taken
+    ActReq* areq;         // [kMaxActSlots]
     int* flag;
     uint32_t* tag;   // [1] this launch's score tag
     // routing of the batch, identical in every CTA
@@ -206,10 +207,10 @@ __host__ __device__ inline Layout layout_of(const FusedParams& p) {
     L.bias = o; o += a16(sizeof(float) * p.E);
     L.desc = o; o += a16(sizeof(Desc) * p.nstage);
     L.task = o; o += a16(sizeof(Task) * kTaskSlots);
-    L.areq = o; o += a16(sizeof(ActReq) * kActSlots);
+    L.areq = o; o += a16(sizeof(ActReq) * kMaxActSlots);
     L.gbuf = o; o += a16(sizeof(float) * 2 * kTaskSlots * kMaxT * kUgTileRows);
     L.red = o; o += a16(sizeof(double) * kConsumerWarps * kMaxRouterRows * kMaxT);
-    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 4 * kActSlots + 2 * kTaskSlots + 1));
+    L.bars = o; o += a16(sizeof(uint64_t) * (2 * p.nstage + 4 * kMaxActSlots + 2 * kTaskSlots + 1));
     L.misc = o; o += a16(sizeof(int) * (4 + 4 + 5 * kMaxPairs + 2));
     L.total = o;
     return L;
@@ -236,12 +237,12 @@ __device__ Smem carve(uint8_t* base, const FusedParams& p) {
     s.full = reinterpret_cast<uint64_t*>(base + L.bars);
     s.empty = s.full + p.nstage;
     s.afull = s.empty + p.nstage;
-    s.aempty = s.afull + kActSlots;
-    s.tfull = s.aempty + kActSlots;
+    s.aempty = s.afull + kMaxActSlots;
+    s.tfull = s.aempty + kMaxActSlots;
     s.tfree = s.tfull + kTaskSlots;
     s.route_bar = s.tfree + kTaskSlots;
     s.areq_full = s.route_bar + 1;
-    s.areq_free = s.areq_full + kActSlots;
+    s.areq_free = s.areq_full + kMaxActSlots;
     s.flag = reinterpret_cast<int*>(base + L.misc);
     s.tag = reinterpret_cast<uint32_t*>(s.flag + 4);
     s.rt_w = reinterpret_cast<float*>(s.tag + 4);
@@ -251,6 +252,14 @@ __device__ Smem carve(uint8_t* base, const FusedParams& p) {
     s.rt_ptok = s.rt_off + kMaxPairs + 1;
     s.rt_U = s.rt_ptok + kMaxPairs;
     return s;
+}
+
+// Activation-record slot i: the first kActSlots have their own region, the
+// others sit in the x cache (neither x nor the routing scratch is read once
+// the routing is done, and the first record copy follows it).
+__device__ __forceinline__ uint8_t* act_slot(const FusedParams& p, const Smem& s, int i) {
+    return i < kActSlots ? s.act + static_cast<size_t>(i) * p.act_bytes
+                         : reinterpret_cast<uint8_t*>(s.xs) + static_cast<size_t>(i - kActSlots) * p.act_bytes;
 }
 
 template <int QT>
@@ -506,7 +515,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                 ok = issue(d, ex.w_down + r * rb_d, static_cast<uint32_t>(d.nrows * rb_d), ex.s_down + r,
                            static_cast<uint32_t>(d.nrows * 4));
             }
-            if (++aslot == kActSlots) {
+            if (++aslot == p.nact) {
                 aslot = 0;
                 aphase ^= 1u;
             }
@@ -1017,7 +1026,7 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
     const int lane = threadIdx.x & 31;
     const int nbI = p.I / 32;
     const size_t rb = static_cast<size_t>(p.I) * QT / 8;
-    const uint8_t* act = s.act + static_cast<size_t>(d.aslot) * p.act_bytes;
+    const uint8_t* act = act_slot(p, s, d.aslot);
     const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
     const int n_tok = d.n_tok, nrows = d.nrows, row0 = d.row0;
     int pair[NT];
@@ -1178,7 +1187,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                         break;
                     }
                     if constexpr (NT == 1) {
-                        const uint8_t* rec = s.act + static_cast<size_t>(aslot) * p.act_bytes;
+                        const uint8_t* rec = act_slot(p, s, aslot);
                         const int nbI = p.I / 32;
 #pragma unroll
                         for (int j = 0; j < kRegChunksDown; ++j) {
@@ -1199,7 +1208,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                 if (d.sit + kGroups >= d.nst) {
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.aempty[aslot]);
-                    if (++aslot == kActSlots) {
+                    if (++aslot == p.nact) {
                         aslot = 0;
                         aphase ^= 1u;
                     }
@@ -1248,18 +1257,18 @@ __device__ __forceinline__ void helper_warp(const FusedParams& p, const Smem& s)
         }
         fence_proxy_async_global();
         mbar_arrive_expect_tx(&s.afull[slot], rq.bytes);
-        bulk_g2s(s.act + static_cast<size_t>(slot) * p.act_bytes, rq.src, rq.bytes, &s.afull[slot]);
+        bulk_g2s(act_slot(p, s, slot), rq.src, rq.bytes, &s.afull[slot]);
         ++n_act;
         mbar_arrive(&s.areq_free[slot]);
-        if (++slot == kActSlots) {
+        if (++slot == p.nact) {
             slot = 0;
             ph ^= 1u;
         }
     }
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
     // drain: every record copy issued into this CTA's shared memory has landed
-    for (int a = 0; a < kActSlots; ++a) {
-        const long uses = n_act / kActSlots + (a < n_act % kActSlots ? 1 : 0);
+    for (int a = 0; a < p.nact; ++a) {
+        const long uses = n_act / p.nact + (a < n_act % p.nact ? 1 : 0);
         if (uses > 0) mbar_wait(&s.afull[a], static_cast<uint32_t>((uses - 1) & 1), kProducerWait);
     }
 }
@@ -1292,30 +1301,35 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
                                         reinterpret_cast<float*>(rec + p.I) + tk.blk,
                                         reinterpret_cast<int32_t*>(rec + p.I + nbI * 4) + tk.blk);
             }
+            // each lane's record words before the bulk copies (async proxy) that
+            // read them in other CTAs; the warp's writes before lane 0's release;
+            // nothing waits for the count here, so the add does not return
             fence_proxy_async_global();
-            __threadfence();
             __syncwarp();
-            if (lane == 0) atomicAdd(p.ug_done + tk.cslot, 1);
+            if (lane == 0) red_release_add_gpu(p.ug_done + tk.cslot, 1);
         } else {
             // count the down tile for its row block; the CTA completing a block combines it
             const int blk = tk.blk, n_experts = tk.n_experts;
             int last = 0;
-            if (lane == 0) {
-                __threadfence();
-                last = atomicAdd(p.rb_done + blk, 1) == n_experts - 1;
-                if (last) __threadfence();
-            }
+            // release: the consumers' y rows of this tile (ordered before this
+            // warp by the task barrier); acquire: every other tile's rows, for
+            // the CTA that completes the block
+            if (lane == 0) last = atom_add_acq_rel_gpu(p.rb_done + blk, 1) == n_experts - 1;
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
-                const int c0 = blk * p.dr, nr = min(p.dr, p.H - c0);
+                // every load of an element first (they are L2 round trips, at
+                // the end of the launch), then the sum in slot order
+                const int c0 = blk * p.dr, nr = min(p.dr, p.H - c0), K = p.K;
                 for (int i = lane; i < p.T * nr; i += 32) {
                     const int t = i / nr, c = c0 + i % nr;
+                    float yv[kMaxExpertsPerLane];
+#pragma unroll
+                    for (int k = 0; k < kMaxExpertsPerLane; ++k)
+                        yv[k] = k < K ? __ldcg(p.y + static_cast<size_t>(s.rt_pair_of[t * K + k]) * p.H + c) : 0.0f;
                     float o = p.has_shared ? __ldcg(p.y + static_cast<size_t>(P + t) * p.H + c) : 0.0f;
-                    for (int k = 0; k < p.K; ++k) {
-                        const int pr = s.rt_pair_of[t * p.K + k];
-                        const float wk = s.rt_w[t * p.K + k];
-                        o = __fadd_rn(o, __fmul_rn(wk, __ldcg(p.y + static_cast<size_t>(pr) * p.H + c)));
-                    }
+#pragma unroll
+                    for (int k = 0; k < kMaxExpertsPerLane; ++k)
+                        if (k < K) o = __fadd_rn(o, __fmul_rn(s.rt_w[t * K + k], yv[k]));
                     if (p.out_bf16) {
                         static_cast<uint16_t*>(p.out)[static_cast<size_t>(t) * p.H + c] = f32_to_bf16_bits(o);
                     } else {
@@ -1349,7 +1363,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], kGroupWarps);
         }
-        for (int i = 0; i < kActSlots; ++i) {
+        for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.afull[i], 1);
             mbar_init(&s.aempty[i], kConsumerWarps);
         }
@@ -1358,7 +1372,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfree[i], 1);
         }
         mbar_init(s.route_bar, 1);
-        for (int i = 0; i < kActSlots; ++i) {
+        for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.areq_full[i], 1);
             mbar_init(&s.areq_free[i], 1);
         }
@@ -1426,6 +1440,10 @@ bool fused_geometry(FusedParams& p, int qtype) {
     p.n_dt = (p.H + p.dr - 1) / p.dr;
     p.rec_bytes = static_cast<int>(fused_record_bytes(p.I));
     p.act_bytes = static_cast<int>(a16(static_cast<size_t>(p.T) * p.rec_bytes));
+    {
+        const size_t xs_bytes = a16(std::max(static_cast<size_t>(p.T) * p.H * 2, sizeof(RouteScratch)));
+        p.nact = kActSlots + static_cast<int>(std::min<size_t>(kMaxActSlots - kActSlots, xs_bytes / p.act_bytes));
+    }
     const bool regs_fit = p.H / 32 <= 32 * kRegChunksUg && p.I / 32 <= 32 * kRegChunksDown;
     p.nt = (p.T == 1 && regs_fit) ? 1 : kMaxT;
     const size_t cap = 227 * 1024;

@@ -110,6 +110,7 @@ struct FusedParams {
     float* y;       // [(T*K + T)][H] per-pair expert outputs (shared rows last)
     int rec_bytes;
     int nstage, stage_bytes, act_bytes, sr_down, dr, n_ugt, n_dt;
+    int nact;  // activation-record slots (2 of their own, the rest in the x cache)
     int rps;   // router rows per stage
     int n_rt;  // router tickets
     int nt;    // token capacity of the kernel instantiation (1 or kFusedMaxTokens)

@@ -128,6 +128,14 @@ __device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
     asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Atomic add returning the old value, with acquire and release semantics at
+// GPU scope: one round trip instead of a fence, the add and another fence.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
 // Polls *p until it reaches `target`, then orders later loads after it
 // (relaxed polls and one fence: an acquire load per poll would invalidate the
 // SM's L1 every time); false after `limit` polls.
