@@ -538,22 +538,51 @@ def run_cuda(args):
     L.moe_profile_read(ctypes.byref(kms), ctypes.byref(kn))
     L.moe_profile_enable(0)
 
-    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region.
+    # Each step copies its own token host -> device and its output row device -> host.  The
+    # copies run on two side streams ordered by events (inputs and outputs double-buffered):
+    # step i + 1's input crosses while step i computes, and the layer kernels stay back to
+    # back on the compute stream.
     x_host = torch.from_numpy(pool.view(np.int16)).view(torch.bfloat16).pin_memory()
-    out_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
     e2e_steps = max(min(args.steps, 3000), 1000)
+    out_host = torch.empty(e2e_steps, T, H, dtype=torch.bfloat16).pin_memory()
+    x_db = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    o_db = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def h2d(i):
+        b = i % 2
+        j = (args.warmup + i) % args.pool
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[b])  # step i - 2 has read x_db[b]
+            x_db[b].copy_(x_host[j:j + 1], non_blocking=True)
+            ev_in[b].record(s_in)
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    h2d(0)
     for i in range(e2e_steps):
-        j = (args.warmup + i) % args.pool
+        b = i % 2
         d = devs[i % NL]
-        x_dev.copy_(x_host[j:j + 1], non_blocking=True)
-        moe.moe_layer_forward(x_dev, d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], out, ws)
-        out_host.copy_(out, non_blocking=True)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])  # step i - 2's output has left o_db[b]
+        moe.moe_layer_forward(x_db[b], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], o_db[b], ws)
+        ev_done[b].record(stream)
+        if i + 1 < e2e_steps:
+            h2d(i + 1)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            out_host[i].copy_(o_db[b], non_blocking=True)
+            ev_out[b].record(s_out)
+    stream.wait_event(ev_out[(e2e_steps - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -608,7 +637,8 @@ def run_cuda(args):
                      "frac": (dom_gbs / hbm_peak) if dom_gbs else None, "traffic": profiled_traffic(),
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
         "e2e": {"value": replicas_tokens_per_s(world, T, e2e_steps, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps},
+                "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps,
+                "copies": "one per step each way, on side streams ordered by events, double-buffered"},
         "gpu_launches": int(launches),
         "clocks": clocks,
         "wall_s_timed_region": wall,

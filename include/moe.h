@@ -284,6 +284,19 @@ int moe_layer_path(int T, const moe_router_cfg* cfg, const moe_experts* routed, 
  */
 int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream);
 
+/*
+ * Test and diagnosis only.  From the next call on `ws` (in stream order), every
+ * bounded device-side wait of moe_layer_forward's kernels gives up after at
+ * most `polls` polls (0 restores the defaults: about a second for each wait)
+ * and records MOE_EDEVICE_TIMEOUT; the kernels then stop issuing work, let
+ * the copies already in flight land (those last waits keep their defaults),
+ * release what they hold and exit, leaving the output unspecified.  A status
+ * clear (moe_workspace_status with `clear` != 0) also restores the defaults.
+ * Writes one word of the library-owned header of `ws` on `stream`; returns
+ * MOE_OK, MOE_EINVAL (null ws, polls < 0) or MOE_ECUDA.
+ */
+int moe_workspace_set_wait_limit(void* ws, int polls, moe_stream_t stream);
+
 /* ------------------------------------------------------------ measurement */
 
 /*

@@ -2,6 +2,7 @@
 // carving and the launch sequence of each call.  No device memory is
 // allocated here; every scratch buffer is carved from the caller's workspace.
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -430,6 +431,7 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
         gp.pair_tok = L.pair_tok;
         gp.pair_slot = L.pair_slot;
         gp.status = L.status;
+        gp.wait_limit = &reinterpret_cast<const FusedSync*>(reinterpret_cast<const uint8_t*>(L.status) + kWsSyncOff)->wait_limit;
         GemmOperands go{};
         go.n_expert = E;
         // up/gate: Q8_0(h) per pair (union order), shared rows last
@@ -521,6 +523,17 @@ int moe_profile_read(double* total_ms, int* launches) {
 }
 
 long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int moe_workspace_set_wait_limit(void* ws, int polls, moe_stream_t stream) {
+    NvtxRange nvtx("moe_workspace_set_wait_limit");
+    if (!ws || polls < 0) return MOE_EINVAL;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int32_t v = polls;  // pageable source: copied out before the call returns
+    const size_t off = kWsSyncOff + offsetof(FusedSync, wait_limit);
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(ws) + off, &v, sizeof(v), cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return MOE_ECUDA;
+    return MOE_OK;
+}
 
 int moe_workspace_status(void* ws, int clear, int* status, moe_stream_t stream) {
     NvtxRange nvtx("moe_workspace_status");

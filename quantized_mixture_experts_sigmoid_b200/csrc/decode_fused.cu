@@ -86,6 +86,8 @@ constexpr int kRegChunksDown = 2;    // NT = 1: blocks of h per lane held in reg
 constexpr long kProducerWait = 1L << 22;
 constexpr long kConsumerWait = 1L << 24;
 constexpr long kEpilogueWait = 1L << 25;
+// (The drains that wait for this CTA's own copies in flight keep kProducerWait
+// whatever the test limit below says: a copy may not land after the exit.)
 constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps (group g: 2 + g)
 constexpr int kBarAfterDep = 4;      // all warps but the producer, after the grid dependency
 static_assert(kStageRows == 2 * kGroupWarps, "an up/gate stage gives each warp of a group two rows");
@@ -262,6 +264,13 @@ __device__ __forceinline__ uint8_t* act_slot(const FusedParams& p, const Smem& s
                          : reinterpret_cast<uint8_t*>(s.xs) + static_cast<size_t>(i - kActSlots) * p.act_bytes;
 }
 
+// Poll limit of a wait: its default, or the workspace's test limit when that
+// is set (nonzero) and smaller (see moe_workspace_set_wait_limit).
+__device__ __forceinline__ long lim(const Smem& s, long dflt) {
+    const long k = s.flag[2];
+    return k > 0 && k < dflt ? k : dflt;
+}
+
 template <int QT>
 __device__ __forceinline__ WBlock<QT> load_wblock_smem(const uint8_t* row, int b) {
     WBlock<QT> r;
@@ -357,10 +366,10 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
         if (n_issued >= kMaxInflight) {  // at most kMaxInflight copies in flight
             const long older = n_issued - kMaxInflight;
             if (!mbar_wait(&s.full[older % p.nstage], static_cast<uint32_t>((older / p.nstage) & 1),
-                           kProducerWait))
+                           lim(s, kProducerWait)))
                 return false;
         }
-        return mbar_wait(&s.empty[stage], sphase ^ 1u, kProducerWait);
+        return mbar_wait(&s.empty[stage], sphase ^ 1u, lim(s, kProducerWait));
     };
     auto advance = [&]() {
         ++n_issued;
@@ -432,7 +441,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
             kind = 0; u = -1; j = t;
         } else {
             if (U < 0) {
-                if (!mbar_wait(s.route_bar, 0, kProducerWait)) {
+                if (!mbar_wait(s.route_bar, 0, lim(s, kProducerWait))) {
                     ok = false;
                     break;
                 }
@@ -490,7 +499,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                   // weight stages stream meanwhile
             d.type = D_DOWN;
             d.mat = 2;
-            if (!mbar_wait(&s.areq_free[aslot], aphase ^ 1u, kProducerWait)) {
+            if (!mbar_wait(&s.areq_free[aslot], aphase ^ 1u, lim(s, kProducerWait))) {
                 ok = false;
                 break;
             }
@@ -524,7 +533,7 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
     if (!ok) record_status(p.status, MOE_EDEVICE_TIMEOUT);
     if (!marked) mark();  // the consumers route before they look for the end
     // tell the helper warp and the consumers to stop
-    if (mbar_wait(&s.areq_free[aslot], aphase ^ 1u, kProducerWait)) {
+    if (mbar_wait(&s.areq_free[aslot], aphase ^ 1u, lim(s, kProducerWait))) {
         s.areq[aslot].exit = 1;
         mbar_arrive(&s.areq_full[aslot]);
     }
@@ -765,7 +774,7 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
                     sc = __uint_as_float(static_cast<uint32_t>(v));
                     break;
                 }
-                if (it >= kConsumerWait) {
+                if (it >= lim(s, kConsumerWait)) {
                     ok = false;
                     break;
                 }
@@ -1094,7 +1103,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     uint32_t tph[kTaskSlots] = {0, 0};
     // Waits for the current stage; returns its type (D_EXIT on timeout).
     auto next_type = [&]() -> int {
-        if (!mbar_wait(&s.full[stage], phase, kConsumerWait)) {
+        if (!mbar_wait(&s.full[stage], phase, lim(s, kConsumerWait))) {
             record_status(p.status, MOE_EDEVICE_TIMEOUT);
             return D_EXIT;
         }
@@ -1111,7 +1120,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     };
     // Waits until epilogue warp tb has finished with task slot tb.
     auto task_slot_free = [&]() -> bool {
-        if (!mbar_wait(&s.tfree[tb], tph[tb] ^ 1u, kConsumerWait)) {
+        if (!mbar_wait(&s.tfree[tb], tph[tb] ^ 1u, lim(s, kConsumerWait))) {
             record_status(p.status, MOE_EDEVICE_TIMEOUT);
             return false;
         }
@@ -1181,7 +1190,7 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                 const Desc& d = s.desc[stage];
                 const uint8_t* sbuf = s.ring + stage * slot_bytes;
                 if (d.sit < kGroups) {
-                    if (!mbar_wait(&s.afull[aslot], aphase, kConsumerWait)) {
+                    if (!mbar_wait(&s.afull[aslot], aphase, lim(s, kConsumerWait))) {
                         record_status(p.status, MOE_EDEVICE_TIMEOUT);
                         ok = false;
                         break;
@@ -1244,14 +1253,14 @@ __device__ __forceinline__ void helper_warp(const FusedParams& p, const Smem& s)
     uint32_t ph = 0;
     bool ok = true;
     while (true) {
-        if (!mbar_wait(&s.areq_full[slot], ph, kProducerWait)) {
+        if (!mbar_wait(&s.areq_full[slot], ph, lim(s, kProducerWait))) {
             ok = false;
             break;
         }
         const ActReq rq = s.areq[slot];
         if (rq.exit) break;
-        if (!mbar_wait(&s.aempty[slot], ph ^ 1u, kProducerWait) ||
-            !wait_counter_geq(p.ug_done + rq.cslot, rq.need, kProducerWait)) {
+        if (!mbar_wait(&s.aempty[slot], ph ^ 1u, lim(s, kProducerWait)) ||
+            !wait_counter_geq(p.ug_done + rq.cslot, rq.need, lim(s, kProducerWait))) {
             ok = false;
             break;
         }
@@ -1282,7 +1291,7 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
     const int P = p.T * p.K;
     uint32_t eph = 0;
     while (true) {
-        if (!mbar_wait(&s.tfull[tb], eph, kEpilogueWait)) {
+        if (!mbar_wait(&s.tfull[tb], eph, lim(s, kEpilogueWait))) {
             record_status(p.status, MOE_EDEVICE_TIMEOUT);
             break;
         }
@@ -1372,6 +1381,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfree[i], 1);
         }
         mbar_init(s.route_bar, 1);
+        s.flag[2] = ld_relaxed_gpu(&p.sync->wait_limit);  // set by the host before the launch
         for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.areq_full[i], 1);
             mbar_init(&s.areq_free[i], 1);

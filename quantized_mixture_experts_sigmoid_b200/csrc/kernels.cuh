@@ -69,7 +69,8 @@ constexpr int kFusedMaxTokens = 4;
 struct FusedSync {
     int ticket;
     int exit_count;
-    int pad[14];
+    int wait_limit;  // test knob: nonzero caps every bounded wait at that many polls
+    int pad[13];
 };
 constexpr size_t kWsStatusOff = 0;
 constexpr size_t kWsSyncOff = 64;
@@ -142,6 +143,7 @@ struct GemmParams {
     float* y;                // down out: routed [T][K][H]
     float* ys;               //           shared [T][H]
     int32_t* status;
+    const int32_t* wait_limit;  // the workspace header's test limit on pipeline waits
 };
 
 struct GemmOperands {

@@ -99,12 +99,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 // Pipeline wait: polls without sleeping (try_wait suspends in hardware), so a
-// phase that completes is seen at once; gives up after kGemmWaitNs.
-__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, int32_t* status) {
+// phase that completes is seen at once; gives up after kGemmWaitNs, or after
+// `polls` polls when the workspace's test limit is set (nonzero).
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, int32_t* status, uint32_t polls) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (polls != 0 && i >= polls) break;
         if ((i & 255u) == 0 && globaltimer_ns() - t0 > kGemmWaitNs) break;
     }
     record_status(status, MOE_EDEVICE_TIMEOUT);
@@ -217,6 +219,8 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                const __grid_constant__ CUtensorMap tm_b0s, const __grid_constant__ CUtensorMap tm_b1s) {
     extern __shared__ __align__(1024) uint8_t gsm_raw[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the workspace's test limit on pipeline waits (0: none; the final drains ignore it)
+    const uint32_t wl = static_cast<uint32_t>(ld_relaxed_gpu(p.wait_limit));
     GemmSmem s;
     {
         const uintptr_t base = (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~static_cast<uintptr_t>(1023);
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                     if (ks >= ksteps || !ok) continue;
                     const float2 dk = dq[j];
                     if (ks + kPre < ksteps) dq[j] = __ldg(d2 + ks + kPre);
-                    if (!gwait(&s.empty[stage], phase, p.status)) {
+                    if (!gwait(&s.empty[stage], phase, p.status, wl)) {
                         ok = false;
                         continue;
                     }
@@ -409,7 +413,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 const CUtensorMap* b1 = it.shared ? &tm_b1s : &tm_b1;
                 const int wr = (it.shared ? 0 : it.e * nout) + nt * cols_per_tile;
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    if (!gwait(&s.empty[stage], phase ^ 1u, p.status)) {
+                    if (!gwait(&s.empty[stage], phase ^ 1u, p.status, wl)) {
                         ok = false;
                         break;
                     }
@@ -455,11 +459,11 @@ __global__ void __launch_bounds__(kThreadsG, 1)
                 const uint64_t bdesc0 = umma_desc_sw128(s.stage + kTileBytes, 0);
                 for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                     for (int ks = 0; ks < ksteps && ok; ++ks) {
-                        if (!gwait(&s.full[stage], phase, p.status) || !gwait(&s.bready[stage], phase, p.status)) {
+                        if (!gwait(&s.full[stage], phase, p.status, wl) || !gwait(&s.bready[stage], phase, p.status, wl)) {
                             ok = false;
                             break;
                         }
-                        if (!gwait(&s.rempty[pair], rphase ^ 1u, p.status)) {
+                        if (!gwait(&s.rempty[pair], rphase ^ 1u, p.status, wl)) {
                             ok = false;
                             break;
                         }
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(kThreadsG, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
                 for (int ks = 0; ks < ksteps; ++ks) {
-                    if (!gwait(&s.full[stage], phase, p.status)) {
+                    if (!gwait(&s.full[stage], phase, p.status, wl)) {
                         ok = false;
                         break;
                     }

@@ -89,7 +89,7 @@ EXPORTS = ["moe_strerror", "moe_route_workspace_bytes", "moe_route", "moe_union"
            "moe_quantize_q8_0", "moe_expert_ffn_workspace_bytes", "moe_expert_ffn_q",
            "moe_combine", "moe_layer_workspace_bytes", "moe_layer_forward",
            "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count",
-           "moe_route_noalloc", "moe_layer_path", "moe_cuda_error_string"]
+           "moe_route_noalloc", "moe_layer_path", "moe_cuda_error_string", "moe_workspace_set_wait_limit"]
 
 
 def lib() -> ctypes.CDLL:
@@ -122,6 +122,7 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_path.restype = i
     L.moe_layer_forward.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.moe_workspace_status.argtypes = [vp, i, vp, vp]
+    L.moe_workspace_set_wait_limit.argtypes = [vp, i, vp]
     L.moe_profile_enable.argtypes = [i]
     L.moe_profile_read.argtypes = [vp, vp]
     L.moe_launch_count.argtypes = []
@@ -242,6 +243,11 @@ def moe_layer_forward(x, w_router, bias, cfg: RouterCfg, routed: ExpertSet,
         _ptr(x), T, _ptr(w_router), _ptr(bias), ctypes.byref(cfg), ctypes.byref(rs),
         ctypes.byref(ss) if ss is not None else None, _ptr(out), dt, _ptr(topk_idx), _ptr(topk_w),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_workspace_set_wait_limit(ws, polls: int, stream=None) -> None:
+    """Test knob: cap every bounded device wait of later calls on `ws` at `polls` polls (0: defaults)."""
+    _ok("moe_workspace_set_wait_limit", lib().moe_workspace_set_wait_limit(_ptr(ws), int(polls), _stream(stream)))
 
 
 def moe_workspace_status(ws, clear: bool = True, stream=None) -> int:

@@ -139,3 +139,10 @@ def test_layer_path_query():
     small = _cfg(E=16, G=4, TG=2, K=2)
     assert path(4, cfg=small, rr=_ex(n=16)) == moe.PATH_GENERAL  # groups of 4 experts: no fused kernel
     assert path(0) == moe.MOE_EINVAL
+
+
+def test_wait_limit_knob_rejects_bad_arguments_without_a_gpu():
+    # host-side argument checks: nothing is written or launched
+    L = moe.lib()
+    assert L.moe_workspace_set_wait_limit(None, 1, None) == moe.MOE_EINVAL
+    assert L.moe_workspace_set_wait_limit(ctypes.c_void_p(1 << 20), -1, None) == moe.MOE_EINVAL
