@@ -85,12 +85,22 @@ static float sigmoid_f32(float l) { return (float)(1.0 / (1.0 + exp(-(double)l))
  * gap_expert[t] (optional) = b of the last chosen expert minus the best b left
  * among kept groups' experts; gap_group[t] = score of the last kept group
  * minus the best score of a dropped group (INFINITY where nothing is left).
+ *
+ * Adaptive expert top-p ([HN] options list, "--topp 0.7": adaptive expert
+ * top-p with 30-40% less expert traffic; the pages name it and give no
+ * definition).  Reading, applied when 0 < top_p < 1 (any other value leaves
+ * the routing as above): order the K slots by s, largest first (ties: the
+ * earlier slot); keep the shortest such prefix whose running sum of s reaches
+ * top_p times the sum of all K scores, both sums in fp64 (S in slot order,
+ * the running sum in that order); the kept slots stay in slot order at the
+ * front, the others become empty (index -1, weight 0); the gate weights are
+ * renormalised over the kept slots as above (fp32 sum in slot order).
  */
-int oracle_select(const float* logits, int T, const float* bias, int E, int n_group,
-                  int topk_group, int top_k, float rsf, int32_t* topk_idx, float* topk_w,
-                  float* gap_expert, float* gap_group) {
+int oracle_select_topp(const float* logits, int T, const float* bias, int E, int n_group,
+                       int topk_group, int top_k, float rsf, float top_p, int32_t* topk_idx,
+                       float* topk_w, float* gap_expert, float* gap_group) {
     if (T < 0 || E <= 0 || n_group <= 0 || E % n_group != 0 || E / n_group < 2 ||
-        topk_group <= 0 || topk_group > n_group || top_k <= 0 ||
+        topk_group <= 0 || topk_group > n_group || top_k <= 0 || top_k > 32 ||
         top_k > topk_group * (E / n_group))
         return ORACLE_EINVAL;
     const int gsz = E / n_group;
@@ -158,11 +168,36 @@ int oracle_select(const float* logits, int T, const float* bias, int E, int n_gr
                 if (gkeep[e / gsz] && !taken[e] && (!any || b[e] > rest)) { rest = b[e]; any = 1; }
             gap_expert[t] = any ? b[idx[top_k - 1]] - rest : INFINITY;
         }
+        /* adaptive top-p: drop the lowest-s slots past the mass top_p */
+        int kept = top_k;
+        if (top_p > 0.0f && top_p < 1.0f) {
+            int ord[32];
+            for (int k = 0; k < top_k; ++k) {  /* stable insertion sort by s, largest first */
+                int m = k;
+                while (m > 0 && s[idx[ord[m - 1]]] < s[idx[k]]) { ord[m] = ord[m - 1]; --m; }
+                ord[m] = k;
+            }
+            double S = 0.0;
+            for (int k = 0; k < top_k; ++k) S += (double)s[idx[k]];
+            const double thr = (double)top_p * S;
+            double c = 0.0;
+            for (int m = 0; m < top_k; ++m) {
+                c += (double)s[idx[ord[m]]];
+                if (c >= thr) { kept = m + 1; break; }
+            }
+            char keep[32] = {0};
+            for (int m = 0; m < kept; ++m) keep[ord[m]] = 1;
+            int j = 0;
+            for (int k = 0; k < top_k; ++k)
+                if (keep[k]) idx[j++] = idx[k];
+            for (; j < top_k; ++j) idx[j] = -1;
+        }
         /* renormalised, scaled gate weights from the unbiased s */
         float den = 0.0f;
-        for (int k = 0; k < top_k; ++k) den += s[idx[k]];
+        for (int k = 0; k < kept; ++k) den += s[idx[k]];
         float* w = topk_w + (size_t)t * top_k;
         for (int k = 0; k < top_k; ++k) {
+            if (k >= kept) { w[k] = 0.0f; continue; }
             float r = s[idx[k]] / den;
             w[k] = r * rsf;
         }
@@ -171,17 +206,31 @@ int oracle_select(const float* logits, int T, const float* bias, int E, int n_gr
     return 0;
 }
 
-int oracle_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
-                 int E, int n_group, int topk_group, int top_k, float rsf, int32_t* topk_idx,
-                 float* topk_w, float* gap_expert, float* gap_group) {
+int oracle_select(const float* logits, int T, const float* bias, int E, int n_group,
+                  int topk_group, int top_k, float rsf, int32_t* topk_idx, float* topk_w,
+                  float* gap_expert, float* gap_group) {
+    return oracle_select_topp(logits, T, bias, E, n_group, topk_group, top_k, rsf, 0.0f, topk_idx,
+                              topk_w, gap_expert, gap_group);
+}
+
+int oracle_route_topp(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
+                      int E, int n_group, int topk_group, int top_k, float rsf, float top_p,
+                      int32_t* topk_idx, float* topk_w, float* gap_expert, float* gap_group) {
     if (T < 0 || H <= 0 || E <= 0) return ORACLE_EINVAL;
     float* logits = (float*)malloc(sizeof(float) * ((size_t)T * E + 1));
     if (!logits) return ORACLE_ENOMEM;
     oracle_router_logits(x, T, H, w_router, E, logits);
-    int rc = oracle_select(logits, T, bias, E, n_group, topk_group, top_k, rsf, topk_idx, topk_w,
-                           gap_expert, gap_group);
+    int rc = oracle_select_topp(logits, T, bias, E, n_group, topk_group, top_k, rsf, top_p, topk_idx,
+                                topk_w, gap_expert, gap_group);
     free(logits);
     return rc;
+}
+
+int oracle_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
+                 int E, int n_group, int topk_group, int top_k, float rsf, int32_t* topk_idx,
+                 float* topk_w, float* gap_expert, float* gap_group) {
+    return oracle_route_topp(x, T, H, w_router, bias, E, n_group, topk_group, top_k, rsf, 0.0f,
+                             topk_idx, topk_w, gap_expert, gap_group);
 }
 
 /* ----------------------------------------------------------------- union */
@@ -195,6 +244,9 @@ int oracle_route(const uint16_t* x, int T, int H, const float* w_router, const f
  *   offsets[u]  exclusive prefix sum of their counts (n_unique + 1 entries)
  *   pairs       (token, slot) entries grouped by expert ascending, tokens
  *               ascending within an expert; slot = the k with idx[t][k] = e
+ * An index of -1 is an empty slot (dropped by adaptive top-p, or a token the
+ * router could not route) and is left out; any other value outside [0, E)
+ * is an error.
  */
 int oracle_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_unique,
                  int32_t* uniq, int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
@@ -204,6 +256,7 @@ int oracle_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_un
     if (!c) return ORACLE_ENOMEM;
     for (long i = 0; i < (long)T * top_k; ++i) {
         const int e = topk_idx[i];
+        if (e == -1) continue;
         if (e < 0 || e >= E) { free(c); return ORACLE_EINVAL; }
         c[e]++;
     }
@@ -414,6 +467,7 @@ int oracle_expert_ffn_per_token(const oracle_experts* ex, const uint16_t* x, int
     for (int t = 0; t < T; ++t) {
         token_f32(x, H, t, xt);
         for (int k = 0; k < top_k; ++k) {
+            if (topk_idx[(size_t)t * top_k + k] == -1) continue;  /* empty slot */
             int rc = oracle_expert_token(ex, topk_idx[(size_t)t * top_k + k], xt,
                                          y_pairs + ((size_t)t * top_k + k) * H, NULL);
             if (rc) { free(xt); return rc; }
@@ -430,7 +484,8 @@ int oracle_expert_ffn_per_token(const oracle_experts* ex, const uint16_t* x, int
  * expert) and the scaling factor: out[t] = shared(x_t) + sum_k w[t][k] * y_k,
  * the shared expert added with weight 1, accumulated in fp32 in slot order
  * starting from the shared output, then narrowed to bf16 (round to nearest
- * even).  shared_y may be NULL (no shared expert).
+ * even).  shared_y may be NULL (no shared expert).  A slot of weight 0 (an
+ * empty slot) adds nothing: its y is not read.
  */
 void oracle_combine(const float* y_pairs, const float* topk_w, const float* shared_y, int T,
                     int top_k, int H, float* out_f32, uint16_t* out_bf16) {
@@ -438,7 +493,9 @@ void oracle_combine(const float* y_pairs, const float* topk_w, const float* shar
         for (int c = 0; c < H; ++c) {
             float o = shared_y ? shared_y[(size_t)t * H + c] : 0.0f;
             for (int k = 0; k < top_k; ++k) {
-                const float p = topk_w[(size_t)t * top_k + k] * y_pairs[((size_t)t * top_k + k) * H + c];
+                const float wk = topk_w[(size_t)t * top_k + k];
+                if (wk == 0.0f) continue;
+                const float p = wk * y_pairs[((size_t)t * top_k + k) * H + c];
                 o = o + p;
             }
             if (out_f32) out_f32[(size_t)t * H + c] = o;
@@ -449,15 +506,15 @@ void oracle_combine(const float* y_pairs, const float* topk_w, const float* shar
 /* ------------------------------------------------------------------ layer */
 
 /* The whole layer: route, union, routed experts, shared expert, combine. */
-int oracle_layer_forward(const uint16_t* x, int T, const float* w_router, const float* bias,
-                         int E, int n_group, int topk_group, int top_k, float rsf,
-                         const oracle_experts* routed, const oracle_experts* shared,
-                         float* out_f32, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w) {
+int oracle_layer_forward_topp(const uint16_t* x, int T, const float* w_router, const float* bias,
+                              int E, int n_group, int topk_group, int top_k, float rsf, float top_p,
+                              const oracle_experts* routed, const oracle_experts* shared,
+                              float* out_f32, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w) {
     const int H = routed->H;
     if (T < 0 || routed->n_expert != E || (shared && (shared->H != H || shared->n_expert < 1)))
         return ORACLE_EINVAL;
-    int rc = oracle_route(x, T, H, w_router, bias, E, n_group, topk_group, top_k, rsf, topk_idx,
-                          topk_w, NULL, NULL);
+    int rc = oracle_route_topp(x, T, H, w_router, bias, E, n_group, topk_group, top_k, rsf, top_p,
+                               topk_idx, topk_w, NULL, NULL);
     if (rc) return rc;
     const size_t P = (size_t)T * top_k;
     int32_t* uniq = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
@@ -487,4 +544,12 @@ int oracle_layer_forward(const uint16_t* x, int T, const float* w_router, const 
 done:
     free(uniq); free(offsets); free(ptok); free(pslot); free(y); free(ys); free(xt);
     return rc;
+}
+
+int oracle_layer_forward(const uint16_t* x, int T, const float* w_router, const float* bias,
+                         int E, int n_group, int topk_group, int top_k, float rsf,
+                         const oracle_experts* routed, const oracle_experts* shared,
+                         float* out_f32, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w) {
+    return oracle_layer_forward_topp(x, T, w_router, bias, E, n_group, topk_group, top_k, rsf, 0.0f,
+                                     routed, shared, out_f32, out_bf16, topk_idx, topk_w);
 }

@@ -70,7 +70,9 @@ def lib(variant: str = "") -> ctypes.CDLL:
         L.oracle_router_logits.argtypes = [vp, i, i, vp, i, vp]
         L.oracle_router_logits.restype = None
         L.oracle_select.argtypes = [vp, i, vp, i, i, i, i, f, vp, vp, vp, vp]
+        L.oracle_select_topp.argtypes = [vp, i, vp, i, i, i, i, f, f, vp, vp, vp, vp]
         L.oracle_route.argtypes = [vp, i, i, vp, vp, i, i, i, i, f, vp, vp, vp, vp]
+        L.oracle_route_topp.argtypes = [vp, i, i, vp, vp, i, i, i, i, f, f, vp, vp, vp, vp]
         L.oracle_union.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
         L.oracle_q8_0.argtypes = [vp, i, vp, vp]
         L.oracle_q8_0.restype = None
@@ -83,6 +85,7 @@ def lib(variant: str = "") -> ctypes.CDLL:
         L.oracle_combine.argtypes = [vp, vp, vp, i, i, i, vp, vp]
         L.oracle_combine.restype = None
         L.oracle_layer_forward.argtypes = [vp, i, vp, vp, i, i, i, i, f, vp, vp, vp, vp, vp, vp]
+        L.oracle_layer_forward_topp.argtypes = [vp, i, vp, vp, i, i, i, i, f, f, vp, vp, vp, vp, vp, vp]
         _libs[variant] = L
     return _libs[variant]
 
@@ -154,7 +157,8 @@ def router_logits(x_bf16, W):
     return out
 
 
-def select(logits, bias, n_group, topk_group, top_k, rsf):
+def select(logits, bias, n_group, topk_group, top_k, rsf, top_p=0.0):
+    """-> (idx, w, gap_expert, gap_group); 0 < top_p < 1 applies adaptive top-p (empty slots: -1, 0)."""
     lg = _c(logits, np.float32)
     T, E = lg.shape
     b = _c(bias, np.float32)
@@ -162,13 +166,13 @@ def select(logits, bias, n_group, topk_group, top_k, rsf):
     w = np.empty((T, top_k), dtype=np.float32)
     ge = np.empty(T, dtype=np.float32)
     gg = np.empty(T, dtype=np.float32)
-    _check(lib().oracle_select(_p(lg), T, _p(b), E, n_group, topk_group, top_k, rsf, _p(idx),
-                               _p(w), _p(ge), _p(gg)), "oracle_select")
+    _check(lib().oracle_select_topp(_p(lg), T, _p(b), E, n_group, topk_group, top_k, rsf, top_p,
+                                    _p(idx), _p(w), _p(ge), _p(gg)), "oracle_select")
     return idx, w, ge, gg
 
 
-def route(x_bf16, W, bias, n_group, topk_group, top_k, rsf):
-    """-> (idx [T,K] int32, w [T,K] fp32, gap_expert [T], gap_group [T])."""
+def route(x_bf16, W, bias, n_group, topk_group, top_k, rsf, top_p=0.0):
+    """-> (idx [T,K] int32, w [T,K] fp32, gap_expert [T], gap_group [T]); see select for top_p."""
     x = _c(x_bf16, np.uint16)
     W = _c(W, np.float32)
     b = _c(bias, np.float32)
@@ -178,8 +182,8 @@ def route(x_bf16, W, bias, n_group, topk_group, top_k, rsf):
     w = np.empty((T, top_k), dtype=np.float32)
     ge = np.empty(T, dtype=np.float32)
     gg = np.empty(T, dtype=np.float32)
-    _check(lib().oracle_route(_p(x), T, H, _p(W), _p(b), E, n_group, topk_group, top_k, rsf,
-                              _p(idx), _p(w), _p(ge), _p(gg)), "oracle_route")
+    _check(lib().oracle_route_topp(_p(x), T, H, _p(W), _p(b), E, n_group, topk_group, top_k, rsf,
+                                   top_p, _p(idx), _p(w), _p(ge), _p(gg)), "oracle_route")
     return idx, w, ge, gg
 
 
@@ -265,7 +269,7 @@ def combine(y_pairs, w, shared_y):
 
 
 def layer_forward(x_bf16, W, bias, n_group, topk_group, top_k, rsf, routed: Experts,
-                  shared: Experts | None):
+                  shared: Experts | None, top_p=0.0):
     """-> (out_f32 [T,H], out_bf16 [T,H] uint16, idx [T,K], w [T,K])."""
     x = _c(x_bf16, np.uint16)
     W = _c(W, np.float32)
@@ -278,7 +282,8 @@ def layer_forward(x_bf16, W, bias, n_group, topk_group, top_k, rsf, routed: Expe
     w = np.empty((T, top_k), dtype=np.float32)
     rs = routed.struct()
     ss = shared.struct() if shared is not None else None
-    _check(lib().oracle_layer_forward(_p(x), T, _p(W), _p(b), E, n_group, topk_group, top_k, rsf,
-                                      ctypes.byref(rs), ctypes.byref(ss) if ss is not None else None,
-                                      _p(of), _p(ob), _p(idx), _p(w)), "oracle_layer_forward")
+    _check(lib().oracle_layer_forward_topp(_p(x), T, _p(W), _p(b), E, n_group, topk_group, top_k, rsf,
+                                           top_p, ctypes.byref(rs),
+                                           ctypes.byref(ss) if ss is not None else None,
+                                           _p(of), _p(ob), _p(idx), _p(w)), "oracle_layer_forward")
     return of, ob, idx, w

@@ -199,6 +199,111 @@ def test_select_rejects_bad_configs():
             O.select(lg, b, G, TG, K, 2.5)
 
 
+# -------------------------------------------------------- adaptive top-p
+def _topp_cases():
+    out = []
+    with open(os.path.join(GOLDEN, "topp_hand_cases.txt")) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, cfg, lg, bias, idx, w = [s.strip() for s in line.split("|")]
+            E, G, TG, K, rsf, pp = cfg.split()
+            out.append(dict(name=name, E=int(E), G=int(G), TG=int(TG), K=int(K), rsf=float(rsf), p=float(pp),
+                            logits=np.float32([_SYM[s] for s in lg.split()]),
+                            bias=np.float32([float(b) for b in bias.split()]),
+                            idx=[int(i) for i in idx.split()], w=np.float32([float(v) for v in w.split()])))
+    return out
+
+
+@pytest.mark.parametrize("case", _topp_cases(), ids=lambda c: c["name"])
+def test_topp_hand_worked(case):
+    idx, w, _, _ = O.select(case["logits"][None, :], case["bias"], case["G"], case["TG"], case["K"], case["rsf"],
+                            top_p=case["p"])
+    assert idx[0].tolist() == case["idx"]
+    assert np.array_equal(w[0], case["w"])
+
+
+def _brute_topp(logits, bias, G, TG, K, rsf, p):
+    """The top-p reading written out from its definition over the brute-force selection."""
+    T = logits.shape[0]
+    sel = _brute_select(logits, bias, G, TG, K)
+    idx = np.full((T, K), -1, np.int32)
+    w = np.zeros((T, K), np.float32)
+    pf = float(np.float32(p))
+    for t in range(T):
+        s_all = np.float32(1.0 / (1.0 + np.exp(-logits[t].astype(np.float64))))
+        s = [s_all[e] for e in sel[t]]
+        keep = set(range(K))
+        if 0.0 < pf < 1.0:
+            order = sorted(range(K), key=lambda k: (-float(s[k]), k))
+            total = 0.0
+            for k in range(K):
+                total += float(s[k])
+            run = 0.0
+            for m, k in enumerate(order):
+                run += float(s[k])
+                if run >= pf * total:
+                    keep = set(order[:m + 1])
+                    break
+        kept = [k for k in range(K) if k in keep]
+        den = np.float32(0.0)
+        for k in kept:
+            den = np.float32(den + s[k])
+        for j, k in enumerate(kept):
+            idx[t, j] = sel[t][k]
+            w[t, j] = np.float32(np.float32(s[k] / den) * np.float32(rsf))
+    return idx, w
+
+
+@pytest.mark.parametrize("E,G,TG,K", [(256, 8, 4, 8), (16, 4, 2, 2), (64, 8, 3, 6)])
+@pytest.mark.parametrize("p", [0.3, 0.5, 0.7, 0.9, 0.97])
+def test_topp_matches_brute_force(E, G, TG, K, p):
+    rng = np.random.default_rng(E + K + int(p * 100))
+    logits = (1.57 * rng.standard_normal((400, E))).astype(np.float32)
+    logits[:100] = np.round(logits[:100] * 4) / 4  # ties in s
+    bias = (0.1 * rng.standard_normal(E)).astype(np.float32)
+    idx, w, _, _ = O.select(logits, bias, G, TG, K, 2.5, top_p=p)
+    bi, bw = _brute_topp(logits, bias, G, TG, K, 2.5, p)
+    assert np.array_equal(idx, bi)
+    assert np.array_equal(w.view(np.uint32), bw.view(np.uint32))
+
+
+def test_topp_invariants():
+    rng = np.random.default_rng(31)
+    E, G, TG, K, rsf = 256, 8, 4, 8, 2.5
+    logits = (1.57 * rng.standard_normal((500, E))).astype(np.float32)
+    bias = (0.1 * rng.standard_normal(E)).astype(np.float32)
+    base_i, base_w, _, _ = O.select(logits, bias, G, TG, K, rsf)
+    # outside (0, 1) the routing is untouched, bit for bit
+    for p in (0.0, 1.0, -0.5, 1.5, float("nan")):
+        i, w, _, _ = O.select(logits, bias, G, TG, K, rsf, top_p=p)
+        assert np.array_equal(i, base_i) and np.array_equal(w.view(np.uint32), base_w.view(np.uint32))
+    prev = np.ones(len(logits), int)
+    s = np.float32(1.0 / (1.0 + np.exp(-logits.astype(np.float64))))
+    for p in (1e-6, 0.2, 0.5, 0.7, 0.9, 0.999):
+        i, w, _, _ = O.select(logits, bias, G, TG, K, rsf, top_p=p)
+        kept = (i >= 0).sum(1)
+        assert kept.min() >= 1
+        assert np.all(kept >= prev)  # more mass kept, never fewer experts
+        prev = kept
+        for t in range(len(logits)):
+            n = kept[t]
+            assert np.all(i[t, n:] == -1) and np.all(w[t, n:] == 0.0)
+            # kept experts are a subsequence of the full slot list (slot order kept)
+            pos = [base_i[t].tolist().index(e) for e in i[t, :n]]
+            assert pos == sorted(pos)
+            # the kept mass reaches p, and dropping the smallest kept score would not
+            sk = s[t, i[t, :n]].astype(np.float64)
+            S = s[t, base_i[t]].astype(np.float64).sum()
+            assert sk.sum() >= np.float32(p) * S * (1 - 1e-12)
+            assert sk.sum() - sk.min() < np.float32(p) * S
+            assert abs(float(w[t, :n].astype(np.float64).sum()) - rsf) < 1e-5
+        if p == 1e-6:
+            assert np.all(kept == 1) and np.array_equal(i[:, 0], base_i[np.arange(len(logits)),
+                                                                          np.argmax(s[np.arange(len(logits))[:, None], base_i], 1)])
+
+
 # ----------------------------------------------------------------- union
 def test_union_against_bitmap_brute_force_and_invariants():
     rng = np.random.default_rng(8)
@@ -218,6 +323,44 @@ def test_union_against_bitmap_brute_force_and_invariants():
         assert np.array_equal(un["pair_slot"], order % K)
         assert np.array_equal(un["offsets"], np.concatenate([[0], np.cumsum(bitmap.sum(1)[present])]))
         assert np.all(idx[un["pair_tok"], un["pair_slot"]] == np.repeat(present, np.diff(un["offsets"])))
+
+
+def test_union_leaves_out_empty_slots():
+    # -1 marks an empty slot (top-p drop or an unroutable token): no pair, no count
+    rng = np.random.default_rng(12)
+    T, E, K = 50, 64, 6
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    drop = rng.random((T, K)) < 0.3
+    idx2 = np.where(drop, -1, idx).astype(np.int32)
+    un = O.union(idx2, E)
+    flat = idx2.reshape(-1)
+    valid = np.nonzero(flat >= 0)[0]
+    order = valid[np.argsort(flat[valid], kind="stable")]
+    assert un["offsets"][un["n_unique"]] == len(valid)
+    assert np.array_equal(un["pair_tok"][:len(valid)], order // K)
+    assert np.array_equal(un["pair_slot"][:len(valid)], order % K)
+    assert np.array_equal(un["counts"], np.bincount(flat[valid], minlength=E))
+    with pytest.raises(ValueError):
+        O.union(np.where(drop, -2, idx).astype(np.int32), E)
+
+
+def test_combine_skips_zero_weight_slots():
+    # a zero-weight slot adds nothing and its y is not read (NaN there changes nothing)
+    rng = np.random.default_rng(13)
+    T, K, H = 3, 4, 64
+    y = rng.standard_normal((T, K, H)).astype(np.float32)
+    w = rng.random((T, K)).astype(np.float32)
+    w[:, 2] = 0.0
+    ys = rng.standard_normal((T, H)).astype(np.float32)
+    of, _ = O.combine(y, w, ys)
+    y2 = y.copy()
+    y2[:, 2] = np.nan
+    of2, _ = O.combine(y2, w, ys)
+    assert np.array_equal(of.view(np.uint32), of2.view(np.uint32))
+    ref = ys.copy()
+    for k in (0, 1, 3):
+        ref = (ref + w[:, k:k + 1] * y[:, k]).astype(np.float32)
+    assert np.array_equal(of.view(np.uint32), ref.view(np.uint32))
 
 
 # ------------------------------------------------------------------ Q8_0
