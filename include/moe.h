@@ -77,13 +77,22 @@ typedef enum { MOE_OUT_BF16 = 0, MOE_OUT_F32 = 1 } moe_out_dtype;
 /* noaux_tc router configuration ([HN] "구현된 주요 기능", router bullet).
  * n_expert (E) routed experts in n_group contiguous groups of E/n_group
  * (at least 2 per group); topk_group groups kept; top_k experts chosen.
- * Limits: E <= 1024, n_group <= 32, top_k <= 32. */
+ * Limits: E <= 1024, n_group <= 32, top_k <= 32.
+ * top_p: adaptive expert top-p ([HN] options list, "--topp 0.7": fewer
+ * experts read per token).  When 0 < top_p < 1, of the top_k slots chosen
+ * for a token the shortest set of largest unbiased scores s whose sum (fp64,
+ * running in that order, ties to the earlier slot) reaches top_p times the
+ * sum of all top_k scores (fp64, slot order) is kept; the kept slots keep
+ * their slot order and move to the front, the others become empty slots
+ * (index -1, weight 0), and the weights are renormalised over the kept slots.
+ * Any other value (0, 1, negative, NaN) leaves the routing unchanged. */
 typedef struct {
     int n_expert;
     int n_group;
     int topk_group;
     int top_k;
     float routed_scaling_factor;
+    float top_p;  /* adaptive expert top-p; any value outside (0, 1) turns it off (0 is the default) */
 } moe_router_cfg;
 
 /* A stack of n_expert experts of one shape and qtype, every array contiguous:
@@ -121,11 +130,12 @@ size_t moe_route_workspace_bytes(int T, const moe_router_cfg* cfg);
  *   groups; among their experts keep the top_k largest b; ties go to the lower
  *   index; slot order is descending b.
  *   topk_w[t][k] = s[idx] / sum_k s[idx] * routed_scaling_factor
+ *   then adaptive top-p when cfg->top_p is in (0, 1) (see moe_router_cfg)
  * x: [T][H] bf16; w_router: [E][H] fp32; bias: [E] fp32;
  * topk_idx: [T][top_k] int32 out; topk_w: [T][top_k] fp32 out.
- * A token with a NaN score (NaN in x, w_router or bias) gets index -1 (which
- * moe_union rejects) and weight 0 in every slot, and MOE_EDEVICE_INDEX is
- * recorded in the workspace status word.
+ * A token with a NaN score (NaN in x, w_router or bias) gets index -1 (an
+ * empty slot, which moe_union leaves out) and weight 0 in every slot, and
+ * MOE_EDEVICE_INDEX is recorded in the workspace status word.
  * T = 0 is a no-op.  Errors: MOE_EINVAL, MOE_EWORKSPACE, MOE_ECUDA.
  */
 int moe_route(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
@@ -175,9 +185,13 @@ int moe_route_noalloc(const uint16_t* x, int T, int H, const float* w_router, co
  *   pair_tok, pair_slot       [T*top_k] (token, slot) pairs grouped by expert
  *                             ascending, tokens ascending within an expert
  *   counts (optional, NULL)   [E] entries per expert (all E, zeros included)
- * Entries of uniq / offsets past U are left unspecified.  An index outside
- * [0, E) is skipped and recorded as MOE_EDEVICE_INDEX in `status` (optional
- * device int32, not cleared by this call).  One CTA; no workspace.
+ * Entries of uniq / offsets past U are left unspecified.  An index of -1 is
+ * an empty slot (dropped by top-p, or a token the router could not route)
+ * and has no pair; any other index outside [0, E) is skipped too and recorded
+ * as MOE_EDEVICE_INDEX in `status` (optional device int32, not cleared by
+ * this call).  The offsets[U] valid pairs come first in pair_tok / pair_slot;
+ * the remaining entries of the T*top_k get token 0 and slot -1.  One CTA; no
+ * workspace.
  */
 int moe_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_unique,
               int32_t* uniq, int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
@@ -233,7 +247,8 @@ int moe_expert_ffn_q(const moe_experts* ex, const uint16_t* x, int T, int top_k,
  * shared expert; routed_scaling_factor already inside topk_w).
  *   o[t][c] = shared_y[t][c] + sum_k topk_w[t][k] * y_pairs[t][k][c]
  * accumulated in fp32 in slot order, each product and sum rounded separately;
- * out is fp32 or bf16 (round to nearest even).  shared_y may be NULL.
+ * a slot whose weight is 0 (an empty slot) adds nothing and its y_pairs row is
+ * not read.  out is fp32 or bf16 (round to nearest even).  shared_y may be NULL.
  */
 int moe_combine(const float* y_pairs, const float* topk_w, const float* shared_y, int T,
                 int top_k, int H, void* out, int out_dtype, moe_stream_t stream);

@@ -193,6 +193,7 @@ bool fused_params(FusedParams& f, const LayerWs& L, void* ws, const uint16_t* x,
     f.TG = c.topk_group;
     f.K = c.top_k;
     f.rsf = c.routed_scaling_factor;
+    f.top_p = c.top_p;
     f.w_router = w_router;
     f.bias = bias;
     f.routed = r;

@@ -829,22 +829,58 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
             if (rank < K) h.slot[rank] = e;
         }
         consumers_sync();
-        // slot k of token t: expert and gate weight
+        // slot k of token t: expert and gate weight; with adaptive top-p the
+        // kept slots (every thread of the first K finds the same set) move to
+        // the front in slot order and the rest become empty (-1, weight 0)
         if (tok && e < K) {
             int ex[kMaxExpertsPerLane];
+            float sv[kMaxExpertsPerLane];
 #pragma unroll
-            for (int k = 0; k < kMaxExpertsPerLane; ++k) ex[k] = k < K ? h.slot[k] : 0;
+            for (int k = 0; k < kMaxExpertsPerLane; ++k) {
+                ex[k] = k < K ? h.slot[k] : 0;
+                sv[k] = k < K ? h.sc[ex[k]] : 0.0f;
+            }
+            uint32_t keep = (1u << K) - 1u;
+            if (p.top_p > 0.0f && p.top_p < 1.0f) {
+                double S = 0.0;
+#pragma unroll
+                for (int k = 0; k < kMaxExpertsPerLane; ++k)
+                    if (k < K) S += static_cast<double>(sv[k]);
+                const double thr = static_cast<double>(p.top_p) * S;
+                double c = 0.0;
+                keep = 0u;
+                for (int m = 0; m < K; ++m) {
+                    int j = -1;  // the largest remaining score, the earlier slot on ties
+                    float best = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < kMaxExpertsPerLane; ++k)
+                        if (k < K && !((keep >> k) & 1u) && (j < 0 || sv[k] > best)) {
+                            j = k;
+                            best = sv[k];
+                        }
+                    keep |= 1u << j;
+                    c += static_cast<double>(best);
+                    if (c >= thr) break;
+                }
+            }
             float den = 0.0f, mys = 0.0f;
 #pragma unroll
             for (int k = 0; k < kMaxExpertsPerLane; ++k) {
-                if (k < K) {
-                    const float sk = h.sc[ex[k]];
-                    den = __fadd_rn(den, sk);
-                    if (k == e) mys = sk;
+                if (k < K && ((keep >> k) & 1u)) {
+                    den = __fadd_rn(den, sv[k]);
+                    if (k == e) mys = sv[k];
                 }
             }
-            rs->pe[t * K + e] = h.slot[e];
-            s.rt_w[t * K + e] = __fmul_rn(__fdiv_rn(mys, den), p.rsf);
+            const int nkept = __popc(keep);
+            if ((keep >> e) & 1u) {
+                const int pos = __popc(keep & ((1u << e) - 1u));
+                rs->pe[t * K + pos] = ex[e];
+                s.rt_w[t * K + pos] = __fmul_rn(__fdiv_rn(mys, den), p.rsf);
+            }
+            if (e >= nkept) {
+                rs->pe[t * K + e] = -1;
+                s.rt_w[t * K + e] = 0.0f;
+            }
         }
         if (tok && e == 0) rs->bad[t] = h.nan;
         consumers_sync();
@@ -857,13 +893,16 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
     for (int t = 0; t < T; ++t) bad_tokens |= rs->bad[t] ? 1u << t : 0u;
     if (bad_tokens && lane == 0) record_status(p.status, MOE_EDEVICE_INDEX);
     const int n = T * K;  // <= 32
-    const bool act = lane < n;
-    const int pe = act ? rs->pe[lane] : 0;
-    const float pw = act ? s.rt_w[lane] : 0.0f;
+    const int pe_raw = lane < n ? rs->pe[lane] : -1;
+    const bool act = pe_raw >= 0;  // a pair (empty slots have none)
+    const int pe = act ? pe_raw : 0;
+    const float pw = lane < n ? s.rt_w[lane] : 0.0f;
+    if (lane < n && !act) s.rt_pair_of[lane] = -1;
     if (T == 1) {
-        // one token: K distinct experts; a pair's position is its expert's rank
+        // one token: distinct experts, the kept ones first; a pair's position is its expert's rank
+        const uint32_t valid = __ballot_sync(all, act);
         int pos = 0;
-        for (int k = 0; k < K; ++k) pos += rs->pe[k] < pe;
+        for (int k = 0; k < K; ++k) pos += ((valid >> k) & 1u) && rs->pe[k] < pe;
         if (act) {
             s.rt_ptok[pos] = 0;
             s.rt_pair_of[lane] = pos;
@@ -871,8 +910,8 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
             s.rt_off[pos] = pos;
         }
         if (lane == 0) {
-            *s.rt_U = K;
-            s.rt_off[K] = K;
+            *s.rt_U = __popc(valid);
+            s.rt_off[__popc(valid)] = __popc(valid);
         }
     } else {
         // pair position = number of pairs with a smaller (expert, token)
@@ -880,6 +919,7 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
         const uint32_t same = __match_any_sync(all, act ? pe : -1 - lane);
         const bool first = act && (__ffs(same) - 1 == lane);
         const uint32_t firsts = __ballot_sync(all, first);
+        const uint32_t valid = __ballot_sync(all, act);
         int pos = 0, urank = 0;
         for (int j = 0; j < n; ++j) {
             const int kj = __shfl_sync(all, key, j);
@@ -896,13 +936,13 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
         }
         if (lane == 0) {
             *s.rt_U = __popc(firsts);
-            s.rt_off[__popc(firsts)] = n;
+            s.rt_off[__popc(firsts)] = __popc(valid);
         }
     }
-    if (act && blockIdx.x == 0) {  // the routing the caller can see, written once
+    if (lane < n && blockIdx.x == 0) {  // the routing the caller can see, written once
         const bool bad = (bad_tokens >> (lane / K)) & 1u;
-        p.idx[lane] = bad ? -1 : pe;
-        p.w[lane] = bad ? 0.0f : pw;
+        p.idx[lane] = bad || !act ? -1 : pe;
+        p.w[lane] = bad || !act ? 0.0f : pw;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(s.route_bar);
@@ -1331,14 +1371,17 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
                 const int c0 = blk * p.dr, nr = min(p.dr, p.H - c0), K = p.K;
                 for (int i = lane; i < p.T * nr; i += 32) {
                     const int t = i / nr, c = c0 + i % nr;
+                    // an empty slot (weight 0, no pair) adds nothing
                     float yv[kMaxExpertsPerLane];
 #pragma unroll
                     for (int k = 0; k < kMaxExpertsPerLane; ++k)
-                        yv[k] = k < K ? __ldcg(p.y + static_cast<size_t>(s.rt_pair_of[t * K + k]) * p.H + c) : 0.0f;
+                        yv[k] = k < K && s.rt_w[t * K + k] != 0.0f
+                                    ? __ldcg(p.y + static_cast<size_t>(s.rt_pair_of[t * K + k]) * p.H + c)
+                                    : 0.0f;
                     float o = p.has_shared ? __ldcg(p.y + static_cast<size_t>(P + t) * p.H + c) : 0.0f;
 #pragma unroll
                     for (int k = 0; k < kMaxExpertsPerLane; ++k)
-                        if (k < K) o = __fadd_rn(o, __fmul_rn(s.rt_w[t * K + k], yv[k]));
+                        if (k < K && s.rt_w[t * K + k] != 0.0f) o = __fadd_rn(o, __fmul_rn(s.rt_w[t * K + k], yv[k]));
                     if (p.out_bf16) {
                         static_cast<uint16_t*>(p.out)[static_cast<size_t>(t) * p.H + c] = f32_to_bf16_bits(o);
                     } else {

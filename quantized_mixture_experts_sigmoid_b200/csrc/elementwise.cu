@@ -32,7 +32,8 @@ k_q8_0(const void* __restrict__ v, long nblocks, int8_t* __restrict__ q, float* 
     }
 }
 
-// out[t][c] = shared[t][c] + sum_k w[t][k] * y[t][k][c]; four columns per thread.
+// out[t][c] = shared[t][c] + sum_k w[t][k] * y[t][k][c] in slot order, slots of
+// weight 0 skipped (empty slots: their y is never written); four columns per thread.
 template <bool BF16_OUT>
 __global__ void __launch_bounds__(256)
 k_combine(const float* __restrict__ y, const float* __restrict__ w, const float* __restrict__ sy,
@@ -46,6 +47,7 @@ k_combine(const float* __restrict__ y, const float* __restrict__ w, const float*
                       : make_float4(0.f, 0.f, 0.f, 0.f);
         for (int k = 0; k < K; ++k) {
             const float wk = w[static_cast<size_t>(t) * K + k];
+            if (wk == 0.0f) continue;  // an empty slot: its y is not read
             const float4 yk = reinterpret_cast<const float4*>(y + (static_cast<size_t>(t) * K + k) * H)[c4];
             o.x = __fadd_rn(o.x, __fmul_rn(wk, yk.x));
             o.y = __fadd_rn(o.y, __fmul_rn(wk, yk.y));

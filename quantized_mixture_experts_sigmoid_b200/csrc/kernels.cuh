@@ -86,6 +86,7 @@ struct FusedParams {
     const uint16_t* x;
     int T, H, I, E, G, TG, K;
     float rsf;
+    float top_p;  // adaptive expert top-p (off outside (0, 1))
     const float* w_router;
     const float* bias;
     moe_experts routed;

@@ -61,7 +61,7 @@ constexpr int kSelectWarps = 4;
 // One warp per token.  Shared memory per warp: s[E], b[E].
 __global__ void __launch_bounds__(kSelectWarps * 32)
 k_router_select(const float* __restrict__ logits, int T, const float* __restrict__ bias, int E,
-                int G, int TG, int K, float rsf, int32_t* __restrict__ topk_idx,
+                int G, int TG, int K, float rsf, float top_p, int32_t* __restrict__ topk_idx,
                 float* __restrict__ topk_w, int32_t* status) {
     extern __shared__ float sm[];
     __shared__ int chosen[kSelectWarps][32];
@@ -70,7 +70,7 @@ k_router_select(const float* __restrict__ logits, int T, const float* __restrict
     if (t >= T) return;
     float* s = sm + static_cast<size_t>(warp) * 2 * E;
     const float* lg = logits + static_cast<size_t>(t) * E;
-    select_token_warp([lg](int e) { return lg[e]; }, bias, E, G, TG, K, rsf, s, s + E,
+    select_token_warp([lg](int e) { return lg[e]; }, bias, E, G, TG, K, rsf, top_p, s, s + E,
                       chosen[warp], topk_idx + static_cast<size_t>(t) * K,
                       topk_w + static_cast<size_t>(t) * K, status);
 }
@@ -98,7 +98,8 @@ cudaError_t launch_router_select(const float* logits, int T, const float* bias,
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(k_router_select), smem);
     if (e != cudaSuccess) return e;
     k_router_select<<<(T + kSelectWarps - 1) / kSelectWarps, kSelectWarps * 32, smem, st>>>(
-        logits, T, bias, c.n_expert, c.n_group, c.topk_group, c.top_k, c.routed_scaling_factor, idx, w, status);
+        logits, T, bias, c.n_expert, c.n_group, c.topk_group, c.top_k, c.routed_scaling_factor, c.top_p, idx, w,
+        status);
     return counted(cudaGetLastError());
 }
 

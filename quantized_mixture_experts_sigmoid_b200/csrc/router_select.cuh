@@ -6,7 +6,12 @@
 // b = s + bias (for choosing only); group score = sum of the two largest b of
 // each contiguous group; keep topk_group groups; choose top_k experts by b
 // among kept groups; ties to the lower index; w = s / sum(s) * rsf with the
-// sum in slot order.
+// sum in slot order.  Adaptive expert top-p (same page, options list:
+// "--topp 0.7"), when 0 < top_p < 1: the slots ranked by s (largest first,
+// ties to the earlier slot), the shortest prefix whose fp64 running sum
+// reaches top_p times the fp64 sum of all K scores is kept, in slot order at
+// the front; the other slots become empty (index -1, weight 0) and the
+// weights are renormalised over the kept ones.
 #pragma once
 
 #include "common.cuh"
@@ -18,7 +23,7 @@ namespace moe {
 // (shared, >= K ints) receives the indices for every lane.
 template <typename LogitFn>
 __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __restrict__ bias,
-                                                  int E, int G, int TG, int K, float rsf,
+                                                  int E, int G, int TG, int K, float rsf, float top_p,
                                                   float* s, float* b, int* chosen,
                                                   int32_t* idx, float* w, int32_t* status) {
     const int lane = threadIdx.x & 31;
@@ -33,7 +38,7 @@ __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __
     __syncwarp();
     if (__any_sync(0xffffffffu, nan)) {
         // a NaN score leaves no expert choosable: every slot gets index -1
-        // (which moe_union rejects) and weight 0
+        // (an empty slot) and weight 0, and the status records it
         record_status(status, MOE_EDEVICE_INDEX);
         for (int k = lane; k < K; k += 32) {
             idx[k] = -1;
@@ -92,15 +97,41 @@ __device__ __forceinline__ void select_token_warp(LogitFn logit, const float* __
         __syncwarp();
     }
     if (lane == 0) {
-        // a slot left without an expert (NaN scores) gets index -1, which
-        // moe_union rejects, and weight 0
+        // adaptive top-p: keep the largest scores until their mass reaches top_p
+        uint32_t kept = K >= 32 ? 0xffffffffu : (1u << K) - 1u;
+        if (top_p > 0.0f && top_p < 1.0f) {
+            double S = 0.0;
+            for (int k = 0; k < K; ++k)
+                if (chosen[k] >= 0) S += static_cast<double>(s[chosen[k]]);
+            const double thr = static_cast<double>(top_p) * S;
+            double c = 0.0;
+            kept = 0u;
+            for (int m = 0; m < K; ++m) {
+                int j = -1;  // the largest remaining score, the earlier slot on ties
+                for (int k = 0; k < K; ++k)
+                    if (!((kept >> k) & 1u) && chosen[k] >= 0 && (j < 0 || s[chosen[k]] > s[chosen[j]])) j = k;
+                if (j < 0) break;
+                kept |= 1u << j;
+                c += static_cast<double>(s[chosen[j]]);
+                if (c >= thr) break;
+            }
+        }
+        // a slot left without an expert (NaN scores) or dropped by top-p gets
+        // index -1 (an empty slot) and weight 0; kept slots move to the front
         float den = 0.0f;
         for (int k = 0; k < K; ++k)
-            if (chosen[k] >= 0) den = __fadd_rn(den, s[chosen[k]]);
+            if (((kept >> k) & 1u) && chosen[k] >= 0) den = __fadd_rn(den, s[chosen[k]]);
+        int j = 0;
         for (int k = 0; k < K; ++k) {
             const int e = chosen[k];
-            idx[k] = e;
-            w[k] = e >= 0 ? __fmul_rn(__fdiv_rn(s[e], den), rsf) : 0.0f;
+            if (!((kept >> k) & 1u) || e < 0) continue;
+            idx[j] = e;
+            w[j] = __fmul_rn(__fdiv_rn(s[e], den), rsf);
+            ++j;
+        }
+        for (; j < K; ++j) {
+            idx[j] = -1;
+            w[j] = 0.0f;
         }
     }
     __syncwarp();

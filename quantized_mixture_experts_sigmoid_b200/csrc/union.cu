@@ -6,6 +6,12 @@
 // of the batch is read once and applied to all positions routed to it.  The
 // lists built here let every later kernel walk experts, not tokens.
 //
+// An index of -1 is an empty slot (dropped by adaptive top-p, or a token the
+// router could not route): it has no pair.  Any other index outside [0, E)
+// records MOE_EDEVICE_INDEX and is left out too.  The pair lists hold the
+// valid pairs first (offsets[n_unique] of them); the rest of the T*K entries
+// get token 0, slot -1, so a pass that walks all T*K rows reads valid rows.
+//
 // One CTA: a shared-memory histogram, a block scan for the compacted expert
 // list and CSR offsets, then a stable counting sort of the T*K entries in
 // chunks of 256 tokens, ranked with per-expert token bitmaps so the pair order
@@ -47,7 +53,7 @@ k_union(const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restric
         const int e = idx[i];
         if (e >= 0 && e < E) {
             atomicAdd(&cnt[e], 1);
-        } else {
+        } else if (e != -1) {
             record_status(status, MOE_EDEVICE_INDEX);
         }
     }
@@ -90,6 +96,10 @@ k_union(const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restric
     if (tid == 0) {
         *n_unique = ptot;
         offsets[ptot] = ctot;
+    }
+    for (long i = ctot + tid; i < n; i += kUnionThreads) {
+        pair_tok[i] = 0;
+        pair_slot[i] = -1;
     }
     __syncthreads();
 

@@ -38,7 +38,7 @@ class MoeError(RuntimeError):
 class RouterCfg(ctypes.Structure):
     _fields_ = [("n_expert", ctypes.c_int), ("n_group", ctypes.c_int),
                 ("topk_group", ctypes.c_int), ("top_k", ctypes.c_int),
-                ("routed_scaling_factor", ctypes.c_float)]
+                ("routed_scaling_factor", ctypes.c_float), ("top_p", ctypes.c_float)]
 
 
 class _Experts(ctypes.Structure):

@@ -360,8 +360,8 @@ def test_layer_forward_repeated_calls_reuse_workspace():
 
 def test_route_nan_token_gets_no_expert():
     # a token whose scores are NaN cannot be routed: every slot gets index -1
-    # and weight 0 (moe_union rejects -1), the workspace router records the code,
-    # and the other tokens of the batch are routed as usual
+    # and weight 0 (an empty slot, which moe_union leaves out), the workspace
+    # router records the code, and the other tokens of the batch are routed as usual
     sh = SHAPES["ragged"]
     dev = dict(W=torch.from_numpy(synth.router_weight(sh)).cuda(),
                bias=torch.from_numpy(synth.router_bias(sh)).cuda(),
@@ -385,4 +385,4 @@ def test_route_nan_token_gets_no_expert():
         assert np.array_equal(np.delete(ig, 3, axis=0), idx_o)
         assert np.array_equal(np.delete(wg, 3, axis=0).view(np.uint32), w_o.view(np.uint32))
         g = gpu_union(ig, sh.E)
-        assert g["status"] == moe.MOE_EDEVICE_INDEX
+        assert g["status"] == 0 and 3 not in g["pair_tok"][:g["offsets"][-1]]
