@@ -388,6 +388,58 @@ def verify_measurement(moe, L, device_layer, to_dev_bf16, name: str, n_layers: i
     }
 
 
+def topp_measurement(moe, L, device_layer, to_dev_bf16, top_p: float, n_layers: int = 4, steps: int = 2000):
+    """Decode (T = 1) with adaptive expert top-p next to the same loop without it: tokens/s, the
+    realised experts per token and the bytes the layer streams per token."""
+    import ctypes
+
+    import torch
+    sh = synth.CONFIGS["decode"]
+    devs = [device_layer(sh, layer=l) for l in range(n_layers)]
+    pool = to_dev_bf16(synth.hidden_states(sh, tokens=range(512)))
+    out = torch.empty(1, sh.H, dtype=torch.bfloat16, device="cuda")
+    d0 = devs[0]
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(1, d0["cfg"], d0["routed"], d0["shared"]))
+    res = {}
+    for p in (1.0, top_p):
+        cfgs = [moe.RouterCfg(d["cfg"].n_expert, d["cfg"].n_group, d["cfg"].topk_group, d["cfg"].top_k,
+                              d["cfg"].routed_scaling_factor, p) for d in devs]
+        idx = torch.empty(steps, sh.top_k, dtype=torch.int32, device="cuda")
+
+        def step(i):
+            d = devs[i % n_layers]
+            moe.moe_layer_forward(pool[i % 512:i % 512 + 1], d["W"], d["bias"], cfgs[i % n_layers], d["routed"],
+                                  d["shared"], out, ws, idx[i % steps])
+
+        for i in range(5):
+            step(i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            step(i)
+        e1.record()
+        torch.cuda.synchronize()
+        if moe.moe_workspace_status(ws) != 0:
+            raise RuntimeError("device status error during the top-p measurement")
+        ms = e0.elapsed_time(e1) / steps
+        kept = (idx.cpu().numpy() >= 0).sum(1)
+        tok_bytes = float((kept.mean() + 1) * sh.expert_bytes() + sh.router_bytes())
+        hbm, kind = peaks()
+        res["p1" if p == 1.0 else "topp"] = {
+            "top_p": p, "tokens_per_s": 1.0 / (ms / 1e3), "us_per_token": ms * 1e3,
+            "experts_per_token": float(kept.mean()), "bytes_per_token": tok_bytes,
+            "GBps": tok_bytes / (ms / 1e3) / 1e9, "frac_of_hbm_peak": tok_bytes / (ms / 1e3) / 1e9 / hbm,
+            "peak_kind": kind}
+    del devs, ws
+    torch.cuda.empty_cache()
+    res["workload"] = (f"GLM-5.2 decode (T=1), {n_layers} resident layers rotated, adaptive expert top-p "
+                       f"{top_p} next to the same loop without it")
+    res["bytes_saved"] = 1.0 - res["topp"]["bytes_per_token"] / res["p1"]["bytes_per_token"]
+    res["speedup"] = res["topp"]["tokens_per_s"] / res["p1"]["tokens_per_s"]
+    return res
+
+
 def stacked_measurement(moe, device_layer, to_dev_bf16, name: str, Ts, reps: int = 10):
     """Stacked decode: all 16 layers resident, timed as one sequence of 16 layer calls (a token
     through the stack), fresh seeded hidden states per layer."""
@@ -539,50 +591,57 @@ def run_cuda(args):
     L.moe_profile_enable(0)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the timed region.
-    # Each step copies its own token host -> device and its output row device -> host.  The
-    # copies run on two side streams ordered by events (inputs and outputs double-buffered):
-    # step i + 1's input crosses while step i computes, and the layer kernels stay back to
-    # back on the compute stream.
+    # Each step copies its own token host -> device and its output row device -> host (one
+    # copy each way per step).  The copies run on two side streams, in chunks of C steps
+    # through rings of 2 C buffers: chunk j + 1's inputs cross while chunk j computes, and
+    # the compute stream waits on the side streams once per chunk, so the layer kernels
+    # otherwise run back to back.
     x_host = torch.from_numpy(pool.view(np.int16)).view(torch.bfloat16).pin_memory()
-    e2e_steps = max(min(args.steps, 3000), 1000)
+    C = 8
+    e2e_steps = max(min(args.steps, 3000), 1000) // C * C
     out_host = torch.empty(e2e_steps, T, H, dtype=torch.bfloat16).pin_memory()
-    x_db = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    o_db = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    x_ring = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2 * C)]
+    o_ring = [torch.empty(T, H, dtype=torch.bfloat16, device="cuda") for _ in range(2 * C)]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # chunk's inputs are on the device
+    ev_done = [torch.cuda.Event() for _ in range(2)]  # chunk's layers have run
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # chunk's outputs have left the device
 
-    def h2d(i):
-        b = i % 2
-        j = (args.warmup + i) % args.pool
+    def h2d_chunk(j):
+        b = j % 2
         with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_done[b])  # step i - 2 has read x_db[b]
-            x_db[b].copy_(x_host[j:j + 1], non_blocking=True)
+            if j >= 2:
+                s_in.wait_event(ev_done[b])  # chunk j - 2 has read these buffers
+            for i in range(j * C, (j + 1) * C):
+                r = (args.warmup + i) % args.pool
+                x_ring[i % (2 * C)].copy_(x_host[r:r + 1], non_blocking=True)
             ev_in[b].record(s_in)
 
+    n_chunks = e2e_steps // C
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    h2d(0)
-    for i in range(e2e_steps):
-        b = i % 2
-        d = devs[i % NL]
+    h2d_chunk(0)
+    for j in range(n_chunks):
+        b = j % 2
         stream.wait_event(ev_in[b])
-        if i >= 2:
-            stream.wait_event(ev_out[b])  # step i - 2's output has left o_db[b]
-        moe.moe_layer_forward(x_db[b], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"], o_db[b], ws)
+        if j >= 2:
+            stream.wait_event(ev_out[b])  # chunk j - 2's outputs have left these buffers
+        for i in range(j * C, (j + 1) * C):
+            d = devs[i % NL]
+            moe.moe_layer_forward(x_ring[i % (2 * C)], d["W"], d["bias"], d["cfg"], d["routed"], d["shared"],
+                                  o_ring[i % (2 * C)], ws)
         ev_done[b].record(stream)
-        if i + 1 < e2e_steps:
-            h2d(i + 1)
+        if j + 1 < n_chunks:
+            h2d_chunk(j + 1)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[b])
-            out_host[i].copy_(o_db[b], non_blocking=True)
+            for i in range(j * C, (j + 1) * C):
+                out_host[i].copy_(o_ring[i % (2 * C)], non_blocking=True)
             ev_out[b].record(s_out)
-    stream.wait_event(ev_out[(e2e_steps - 1) % 2])
+    stream.wait_event(ev_out[(n_chunks - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -594,6 +653,7 @@ def run_cuda(args):
     if world == 1 and not args.no_extras:
         extras["verify"] = verify_measurement(moe, L, device_layer, to_dev_bf16, "verify")
         extras["verify_int8"] = verify_measurement(moe, L, device_layer, to_dev_bf16, "verify_int8")
+        extras["decode_topp"] = topp_measurement(moe, L, device_layer, to_dev_bf16, 0.7)
         extras["stacked"] = stacked_measurement(moe, device_layer, to_dev_bf16, "stacked", (1, 8))
         extras["stacked_int2"] = stacked_measurement(moe, device_layer, to_dev_bf16, "stacked_int2", (1,))
     prefill = prefill_measurement(args, moe, L, device_layer, to_dev_bf16) if args.prefill else None
@@ -638,7 +698,7 @@ def run_cuda(args):
                      "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
         "e2e": {"value": replicas_tokens_per_s(world, T, e2e_steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 2, "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps,
-                "copies": "one per step each way, on side streams ordered by events, double-buffered"},
+                "copies": "one per step each way, on side streams in chunks of 8 steps, rings of 16 buffers"},
         "gpu_launches": int(launches),
         "clocks": clocks,
         "wall_s_timed_region": wall,
