@@ -56,6 +56,77 @@ k_router_logits(const uint16_t* __restrict__ x, const float* __restrict__ w, int
     }
 }
 
+// Batches (T >= kTiledMinT): a register-blocked fp64 GEMM.  A CTA computes
+// 64 tokens x 64 experts, each thread 4 x 4 of them; x and W pass through
+// shared memory in chunks of 16 along H, converted to fp64 once (double
+// buffered).  Every logit is accumulated by one thread in ascending h, the
+// order of the plain definition, so the fp64 sum is that of the definition.
+constexpr int kTiledMinT = 32;
+constexpr int kTM = 64, kTN = 64, kKC = 16, kTiledThreads = 256;
+
+__global__ void __launch_bounds__(kTiledThreads)
+k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
+                      float* __restrict__ logits) {
+    __shared__ __align__(16) double xs[2][kKC][kTM];  // [stage][h][token]
+    __shared__ __align__(16) double wsm[2][kKC][kTN]; // [stage][h][expert]
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.x * kTM, e0 = blockIdx.y * kTN;
+    const int ty = tid >> 4, tx = tid & 15;  // tokens 4 ty .. 4 ty + 3, experts 4 tx .. 4 tx + 3
+    // loader: 64 rows x 16 values per operand per chunk; thread tid loads row tid / 4,
+    // values 4 (tid % 4) .. + 3 of x and of W
+    const int lr = tid >> 2, lc = (tid & 3) * 4;
+    const bool xin = t0 + lr < T, win = e0 + lr < E;
+    const uint16_t* xrow = x + static_cast<size_t>(xin ? t0 + lr : 0) * H + lc;
+    const float* wrow = w + static_cast<size_t>(win ? e0 + lr : 0) * H + lc;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    uint2 xr = xin ? __ldg(reinterpret_cast<const uint2*>(xrow)) : make_uint2(0, 0);
+    float4 wr = win ? __ldg(reinterpret_cast<const float4*>(wrow)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int nk = H / kKC;
+    for (int kc = 0; kc < nk; ++kc) {
+        const int st = kc & 1;
+        xs[st][lc + 0][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.x)));
+        xs[st][lc + 1][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.x >> 16)));
+        xs[st][lc + 2][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.y)));
+        xs[st][lc + 3][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.y >> 16)));
+        wsm[st][lc + 0][lr] = static_cast<double>(wr.x);
+        wsm[st][lc + 1][lr] = static_cast<double>(wr.y);
+        wsm[st][lc + 2][lr] = static_cast<double>(wr.z);
+        wsm[st][lc + 3][lr] = static_cast<double>(wr.w);
+        __syncthreads();
+        if (kc + 1 < nk) {  // the next chunk's values, in flight during this chunk's products
+            xr = xin ? __ldg(reinterpret_cast<const uint2*>(xrow + (kc + 1) * kKC)) : make_uint2(0, 0);
+            wr = win ? __ldg(reinterpret_cast<const float4*>(wrow + (kc + 1) * kKC)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kKC; ++k) {
+            const double2 a01 = *reinterpret_cast<const double2*>(&xs[st][k][4 * ty]);
+            const double2 a23 = *reinterpret_cast<const double2*>(&xs[st][k][4 * ty + 2]);
+            const double2 b01 = *reinterpret_cast<const double2*>(&wsm[st][k][4 * tx]);
+            const double2 b23 = *reinterpret_cast<const double2*>(&wsm[st][k][4 * tx + 2]);
+            const double a[4] = {a01.x, a01.y, a23.x, a23.y}, bb[4] = {b01.x, b01.y, b23.x, b23.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], bb[j], acc[i][j]);
+        }
+        // the stage written next iteration was read two chunks ago: one barrier per chunk suffices
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 4 * ty + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e0 + 4 * tx + j;
+            if (e < E) logits[static_cast<size_t>(t) * E + e] = __double2float_rn(acc[i][j]);
+        }
+    }
+}
+
 constexpr int kSelectWarps = 4;
 
 // One warp per token.  Shared memory per warp: s[E], b[E].
@@ -85,6 +156,9 @@ cudaError_t launch_router_logits(const uint16_t* x, int T, int H, const float* w
         k_router_logits<1><<<dim3(gx, T), block, 0, st>>>(x, w, T, H, E, logits);
     } else if (T <= 4) {
         k_router_logits<4><<<dim3(gx, 1), block, 0, st>>>(x, w, T, H, E, logits);
+    } else if (T >= kTiledMinT && H % kKC == 0) {
+        k_router_logits_tiled<<<dim3((T + kTM - 1) / kTM, (E + kTN - 1) / kTN), kTiledThreads, 0, st>>>(
+            x, w, T, H, E, logits);
     } else {
         k_router_logits<8><<<dim3(gx, (T + 7) / 8), block, 0, st>>>(x, w, T, H, E, logits);
     }
