@@ -210,6 +210,29 @@ int moe_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_uniqu
 int moe_quantize_q8_0(const void* v, int in_dtype, int rows, int n, int8_t* q, float* d,
                       moe_stream_t stream);
 
+/* ------------------------------------------------------------ expert usage */
+
+/*
+ * Expert-usage record ([HN] "Learning cache와 하드웨어별 기대치": the engine
+ * records which experts routing picks and pins the most used ones in spare
+ * RAM; [YO] names the STATS / PIN switches).  usage: [E] uint32 device counts
+ * owned by the caller (zero it once; one record per layer); each call adds,
+ * for every (token, slot) of topk_idx [T][top_k], one to usage[idx].  Empty
+ * slots (-1) and indices outside [0, E) add nothing.  Counts wrap at 2^32.
+ * Errors: MOE_EINVAL (sizes, null pointers), MOE_ECUDA.
+ */
+int moe_usage_accumulate(const int32_t* topk_idx, int T, int top_k, int E, uint32_t* usage,
+                         moe_stream_t stream);
+
+/*
+ * The pin order of a usage record: order[r] (device int32 [E]) = the expert of
+ * rank r, most used first, ties to the lower index.  With every expert of a
+ * B200 resident in HBM, this order is what a caller uses to place the hot
+ * experts (the pages' pinning) wherever its memory hierarchy rewards it.
+ * E <= 1024.  Errors: MOE_EINVAL, MOE_ECUDA.
+ */
+int moe_usage_rank(const uint32_t* usage, int E, int32_t* order, moe_stream_t stream);
+
 /* ----------------------------------------------------------------- experts */
 
 /* Bytes of workspace moe_expert_ffn_q needs. */

@@ -287,3 +287,22 @@ def layer_forward(x_bf16, W, bias, n_group, topk_group, top_k, rsf, routed: Expe
                                            ctypes.byref(ss) if ss is not None else None,
                                            _p(of), _p(ob), _p(idx), _p(w)), "oracle_layer_forward")
     return of, ob, idx, w
+
+
+# ------------------------------------------------------------- expert usage
+# [HN] "Learning cache와 하드웨어별 기대치": routed experts are recorded and the
+# most used ones pinned first.  Plain definitions of the record and its order.
+def usage_accumulate(idx, E, usage=None):
+    """usage[e] + number of entries of idx equal to e (entries outside [0, E), such as the
+    empty slot -1, count for nothing)."""
+    u = np.zeros(E, dtype=np.int64) if usage is None else np.array(usage, dtype=np.int64)
+    for e in np.asarray(idx).reshape(-1).tolist():
+        if 0 <= e < E:
+            u[e] += 1
+    return u
+
+
+def usage_rank(usage):
+    """The experts, most used first, ties to the lower index."""
+    u = [int(v) for v in np.asarray(usage).reshape(-1)]
+    return np.array(sorted(range(len(u)), key=lambda e: (-u[e], e)), dtype=np.int32)

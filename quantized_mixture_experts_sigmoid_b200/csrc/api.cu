@@ -367,6 +367,22 @@ int moe_combine(const float* y_pairs, const float* topk_w, const float* shared_y
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int moe_usage_accumulate(const int32_t* topk_idx, int T, int top_k, int E, uint32_t* usage,
+                         moe_stream_t stream) {
+    NvtxRange nvtx("moe_usage_accumulate");
+    if (T < 0 || top_k <= 0 || top_k > 32 || E <= 0 || E > 1024) return MOE_EINVAL;
+    if (T == 0) return MOE_OK;
+    if (!topk_idx || !usage) return MOE_EINVAL;
+    return cuda_rc(launch_usage_accumulate(topk_idx, static_cast<long>(T) * top_k, E, usage,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_usage_rank(const uint32_t* usage, int E, int32_t* order, moe_stream_t stream) {
+    NvtxRange nvtx("moe_usage_rank");
+    if (E <= 0 || E > 1024 || !usage || !order) return MOE_EINVAL;
+    return cuda_rc(launch_usage_rank(usage, E, order, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t moe_layer_workspace_bytes(int T, const moe_router_cfg* cfg, const moe_experts* routed,
                                  const moe_experts* shared) {
     if (T < 0 || check_cfg(cfg) != MOE_OK || !routed || routed->hidden <= 0 || routed->inter <= 0)

@@ -53,6 +53,8 @@ cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const
 cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
                                int top_k, const UnionView& un, float* y_pairs, cudaStream_t st);
 
+cudaError_t launch_usage_accumulate(const int32_t* idx, long n, int E, uint32_t* usage, cudaStream_t st);
+cudaError_t launch_usage_rank(const uint32_t* usage, int E, int32_t* order, cudaStream_t st);
 cudaError_t launch_combine(const float* y, const float* w, const float* shared_y, int T, int K,
                            int H, void* out, int out_dtype, cudaStream_t st);
 

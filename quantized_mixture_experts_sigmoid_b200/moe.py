@@ -89,7 +89,8 @@ EXPORTS = ["moe_strerror", "moe_route_workspace_bytes", "moe_route", "moe_union"
            "moe_quantize_q8_0", "moe_expert_ffn_workspace_bytes", "moe_expert_ffn_q",
            "moe_combine", "moe_layer_workspace_bytes", "moe_layer_forward",
            "moe_workspace_status", "moe_profile_enable", "moe_profile_read", "moe_launch_count",
-           "moe_route_noalloc", "moe_layer_path", "moe_cuda_error_string", "moe_workspace_set_wait_limit"]
+           "moe_route_noalloc", "moe_layer_path", "moe_cuda_error_string", "moe_workspace_set_wait_limit",
+           "moe_usage_accumulate", "moe_usage_rank"]
 
 
 def lib() -> ctypes.CDLL:
@@ -123,6 +124,8 @@ def lib() -> ctypes.CDLL:
     L.moe_layer_forward.argtypes = [vp, i, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, sz, vp]
     L.moe_workspace_status.argtypes = [vp, i, vp, vp]
     L.moe_workspace_set_wait_limit.argtypes = [vp, i, vp]
+    L.moe_usage_accumulate.argtypes = [vp, i, i, i, vp, vp]
+    L.moe_usage_rank.argtypes = [vp, i, vp, vp]
     L.moe_profile_enable.argtypes = [i]
     L.moe_profile_read.argtypes = [vp, vp]
     L.moe_launch_count.argtypes = []
@@ -243,6 +246,17 @@ def moe_layer_forward(x, w_router, bias, cfg: RouterCfg, routed: ExpertSet,
         _ptr(x), T, _ptr(w_router), _ptr(bias), ctypes.byref(cfg), ctypes.byref(rs),
         ctypes.byref(ss) if ss is not None else None, _ptr(out), dt, _ptr(topk_idx), _ptr(topk_w),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_usage_accumulate(topk_idx, E: int, usage, stream=None) -> None:
+    """usage[e] += entries of topk_idx [T][K] routed to e (empty slots add nothing)."""
+    T, K = topk_idx.shape
+    _ok("moe_usage_accumulate", lib().moe_usage_accumulate(_ptr(topk_idx), T, K, int(E), _ptr(usage), _stream(stream)))
+
+
+def moe_usage_rank(usage, order, stream=None) -> None:
+    """order[r] = the expert of rank r in the usage record (most used first, ties to the lower index)."""
+    _ok("moe_usage_rank", lib().moe_usage_rank(_ptr(usage), usage.numel(), _ptr(order), _stream(stream)))
 
 
 def moe_workspace_set_wait_limit(ws, polls: int, stream=None) -> None:

@@ -146,3 +146,13 @@ def test_wait_limit_knob_rejects_bad_arguments_without_a_gpu():
     L = moe.lib()
     assert L.moe_workspace_set_wait_limit(None, 1, None) == moe.MOE_EINVAL
     assert L.moe_workspace_set_wait_limit(ctypes.c_void_p(1 << 20), -1, None) == moe.MOE_EINVAL
+
+
+def test_usage_calls_reject_bad_arguments_without_a_gpu():
+    L = moe.lib()
+    P = ctypes.c_void_p(1 << 20)
+    assert L.moe_usage_accumulate(None, 4, 8, 256, P, None) == moe.MOE_EINVAL
+    assert L.moe_usage_accumulate(P, 4, 8, 2048, P, None) == moe.MOE_EINVAL
+    assert L.moe_usage_accumulate(P, 0, 8, 256, P, None) == moe.MOE_OK  # empty batch: nothing to add
+    assert L.moe_usage_rank(P, 0, P, None) == moe.MOE_EINVAL
+    assert L.moe_usage_rank(None, 256, P, None) == moe.MOE_EINVAL

@@ -363,6 +363,24 @@ def test_combine_skips_zero_weight_slots():
     assert np.array_equal(of.view(np.uint32), ref.view(np.uint32))
 
 
+def test_usage_record_and_rank_hand_worked():
+    # two batches: experts 1 and 2 used 5 times, 0 three times, 3 never; -1 slots ignored
+    u = O.usage_accumulate(np.array([[1, 2], [0, 1], [2, -1]]), 4)
+    u = O.usage_accumulate(np.array([[1, 2, 0], [2, 1, 0], [1, 2, -1]]), 4, u)
+    assert u.tolist() == [3, 5, 5, 0]
+    assert O.usage_rank(u).tolist() == [1, 2, 0, 3]  # the tie 1 / 2 goes to the lower index
+    assert O.usage_rank(np.zeros(5)).tolist() == [0, 1, 2, 3, 4]
+
+
+def test_usage_rank_is_a_permutation_sorted_by_count():
+    rng = np.random.default_rng(14)
+    u = rng.integers(0, 6, 300)
+    order = O.usage_rank(u)
+    assert sorted(order.tolist()) == list(range(300))
+    keys = [(-int(u[e]), int(e)) for e in order]
+    assert keys == sorted(keys)
+
+
 # ------------------------------------------------------------------ Q8_0
 def test_q8_0_grid_values_round_trip_exactly():
     rng = np.random.default_rng(9)
