@@ -368,6 +368,31 @@ float oracle_qdot(const int8_t* wcodes, float w_scale, const int8_t* qa, const f
     return acc * w_scale;
 }
 
+/*
+ * The same dot with grouped weight scales: one scale per `group` consecutive
+ * codes of the row ([MO] "int4 양자화 (Quantization)의 품질 비용": grouped
+ * scales recover most of int4's quality loss; the page gives no layout).
+ * Reading: block b's integer dot is scaled by the product of its activation
+ * scale and its group's weight scale, d_b * s_w[g(b)] rounded once to fp32,
+ * and folded like the per-row dot: one fused multiply-add per block in
+ * ascending order; there is no separate row scale.
+ */
+float oracle_qdot_grouped(const int8_t* wcodes, const float* w_scales, int group, const int8_t* qa,
+                          const float* da, int n) {
+    float acc = 0.0f;
+    for (int b = 0; b < n / 32; ++b) {
+        int32_t isum = 0;
+        for (int i = 32 * b; i < 32 * b + 32; ++i) isum += (int32_t)qa[i] * (int32_t)wcodes[i];
+        const float f = da[b] * w_scales[(32 * b) / group];
+#ifdef ORACLE_FOLD_MULADD
+        acc = acc + (float)isum * f;
+#else
+        acc = fmaf((float)isum, f, acc);
+#endif
+    }
+    return acc;
+}
+
 /* ---------------------------------------------------------------- expert */
 
 static int row_bytes(int qtype, int n) { return n * qtype / 8; }
@@ -384,8 +409,9 @@ static int row_bytes(int qtype, int n) { return n * qtype / 8; }
  * 전략" places it with the dense part).
  */
 int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* y, float* h_out) {
-    const int H = ex->H, I = ex->I, q = ex->qtype;
+    const int H = ex->H, I = ex->I, q = ex->qtype, gs = ex->group;
     if (e < 0 || e >= ex->n_expert || H % 32 || I % 32) return ORACLE_EINVAL;
+    if (gs < 0 || (gs && (gs % 32 || H % gs || I % gs))) return ORACLE_EINVAL;
     if (!ex->w_gate[e] || !ex->w_up[e] || !ex->w_down[e] || !ex->s_gate[e] || !ex->s_up[e] ||
         !ex->s_down[e])
         return ORACLE_EINVAL;
@@ -406,9 +432,11 @@ int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* 
 #pragma omp for schedule(static)
         for (int r = 0; r < I; ++r) {
             oracle_unpack(ex->w_gate[e] + (size_t)r * rb_in, q, H, codes);
-            const float g = oracle_qdot(codes, ex->s_gate[e][r], qa, da, H);
+            const float g = gs ? oracle_qdot_grouped(codes, ex->s_gate[e] + (size_t)r * (H / gs), gs, qa, da, H)
+                               : oracle_qdot(codes, ex->s_gate[e][r], qa, da, H);
             oracle_unpack(ex->w_up[e] + (size_t)r * rb_in, q, H, codes);
-            const float u = oracle_qdot(codes, ex->s_up[e][r], qa, da, H);
+            const float u = gs ? oracle_qdot_grouped(codes, ex->s_up[e] + (size_t)r * (H / gs), gs, qa, da, H)
+                               : oracle_qdot(codes, ex->s_up[e][r], qa, da, H);
 #ifdef ORACLE_SILU_F32
             const float silu = g / (1.0f + expf(-g));  /* variant: fp32 throughout */
 #else
@@ -421,7 +449,8 @@ int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* 
 #pragma omp for schedule(static)
         for (int c = 0; c < H; ++c) {
             oracle_unpack(ex->w_down[e] + (size_t)c * rb_out, q, I, codes);
-            y[c] = oracle_qdot(codes, ex->s_down[e][c], qh, dh, I);
+            y[c] = gs ? oracle_qdot_grouped(codes, ex->s_down[e] + (size_t)c * (I / gs), gs, qh, dh, I)
+                      : oracle_qdot(codes, ex->s_down[e][c], qh, dh, I);
         }
         free(codes);
     }

@@ -35,7 +35,10 @@ extern "C" {
 /* Expert set on the host: per-expert pointer tables so that a caller can
  * supply only the experts it needs (NULL elsewhere).
  * w_gate[e], w_up[e]: [I][H*qtype/8] packed codes; w_down[e]: [H][I*qtype/8];
- * s_gate[e], s_up[e]: [I] fp32 row scales; s_down[e]: [H]. */
+ * s_gate[e], s_up[e]: [I] fp32 row scales; s_down[e]: [H].
+ * group != 0 (grouped scales): one scale per row and group of `group`
+ * consecutive codes along the row instead: s_gate[e], s_up[e]: [I][H/group],
+ * s_down[e]: [H][I/group]. */
 typedef struct {
     int qtype; /* 2, 4 or 8 bits per weight */
     int n_expert;
@@ -47,6 +50,7 @@ typedef struct {
     const float* const* s_gate;
     const float* const* s_up;
     const float* const* s_down;
+    int group; /* 0: per-row scales; else codes per scale group (a multiple of 32) */
 } oracle_experts;
 
 float oracle_bf16_to_f32(uint16_t v);
@@ -74,6 +78,9 @@ void oracle_q8_0(const float* v, int n, int8_t* q, float* d);
 int oracle_unpack(const uint8_t* packed, int qtype, int n, int8_t* codes);
 
 float oracle_qdot(const int8_t* wcodes, float w_scale, const int8_t* qa, const float* da, int n);
+
+float oracle_qdot_grouped(const int8_t* wcodes, const float* w_scales, int group, const int8_t* qa,
+                          const float* da, int n);
 
 int oracle_expert_token(const oracle_experts* ex, int e, const float* x, float* y, float* h_out);
 

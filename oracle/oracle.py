@@ -53,7 +53,7 @@ class _Experts(ctypes.Structure):
     _fields_ = [("qtype", ctypes.c_int), ("n_expert", ctypes.c_int), ("H", ctypes.c_int),
                 ("I", ctypes.c_int), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p), ("s_gate", ctypes.c_void_p),
-                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
+                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p), ("group", ctypes.c_int)]
 
 
 _libs = {}
@@ -79,6 +79,8 @@ def lib(variant: str = "") -> ctypes.CDLL:
         L.oracle_unpack.argtypes = [vp, i, i, vp]
         L.oracle_qdot.argtypes = [vp, f, vp, vp, i]
         L.oracle_qdot.restype = f
+        L.oracle_qdot_grouped.argtypes = [vp, vp, i, vp, vp, i]
+        L.oracle_qdot_grouped.restype = f
         L.oracle_expert_token.argtypes = [vp, i, vp, vp, vp]
         L.oracle_expert_ffn.argtypes = [vp, vp, i, i, i, vp, vp, vp, vp, vp]
         L.oracle_expert_ffn_per_token.argtypes = [vp, vp, i, i, vp, vp]
@@ -107,11 +109,12 @@ class Experts:
     """Host expert set: per-expert arrays (None where not needed).
 
     gate/up[e]: uint8 [I, H*q/8]; down[e]: uint8 [H, I*q/8];
-    s_gate/s_up[e]: fp32 [I]; s_down[e]: fp32 [H].
+    s_gate/s_up[e]: fp32 [I]; s_down[e]: fp32 [H]; with grouped scales (group != 0)
+    s_gate/s_up[e]: fp32 [I, H/group]; s_down[e]: fp32 [H, I/group].
     """
 
-    def __init__(self, qtype, H, I, n_expert):
-        self.qtype, self.H, self.I, self.n = qtype, H, I, n_expert
+    def __init__(self, qtype, H, I, n_expert, group=0):
+        self.qtype, self.H, self.I, self.n, self.group = qtype, H, I, n_expert, group
         self.gate = [None] * n_expert
         self.up = [None] * n_expert
         self.down = [None] * n_expert
@@ -134,7 +137,7 @@ class Experts:
             tabs.append(arr)
         self._tabs = tabs  # keep alive
         s = _Experts(self.qtype, self.n, self.H, self.I,
-                     *[ctypes.cast(t, ctypes.c_void_p) for t in tabs])
+                     *[ctypes.cast(t, ctypes.c_void_p) for t in tabs], self.group)
         self._struct = s
         return s
 
@@ -225,6 +228,14 @@ def qdot(wcodes, w_scale, qa, da, variant: str = ""):
     qa = _c(qa, np.int8)
     da = _c(da, np.float32)
     return lib(variant).oracle_qdot(_p(wc), float(w_scale), _p(qa), _p(da), wc.size)
+
+
+def qdot_grouped(wcodes, w_scales, group, qa, da, variant: str = ""):
+    wc = _c(wcodes, np.int8)
+    ws = _c(w_scales, np.float32)
+    qa = _c(qa, np.int8)
+    da = _c(da, np.float32)
+    return lib(variant).oracle_qdot_grouped(_p(wc), _p(ws), int(group), _p(qa), _p(da), wc.size)
 
 
 def expert_token(ex: Experts, e, x_f32, want_h=False, variant: str = ""):

@@ -13,7 +13,7 @@ from oracle import oracle as O
 
 def oracle_experts(sh: synth.LayerShape, experts, layer: int = 0, shared: bool = False) -> O.Experts:
     """Oracle expert set holding only the listed experts (regenerated from the seed)."""
-    ex = O.Experts(sh.qtype, sh.H, sh.I, 1 if shared else sh.E)
+    ex = O.Experts(sh.qtype, sh.H, sh.I, 1 if shared else sh.E, group=sh.group_size)
     for e in experts:
         sid = synth.SHARED if shared else int(e)
         g, sg = synth.expert_matrix(sh, layer, sid, synth.GATE)

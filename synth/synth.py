@@ -12,7 +12,8 @@ experts in 8 groups, top-8, one shared expert):
   * expert weights: packed int4 / int2 codes are uniform random bytes (every
     nibble / 2-bit field of a uniform byte is uniform over its code range,
     [-8,7] / [-2,1] after the offset); int8 codes are uniform on [-127,127];
-  * per-row scales: U(0.01, 0.05) in fp32;
+  * per-row scales: U(0.01, 0.05) in fp32 (grouped scales, group_size != 0: one
+    per row and group, the same stream read at index row * groups + group);
   * router weight: fp32 N(0, 0.02^2); correction bias: fp32 N(0, 0.1^2),
     plus, for the Zipf-skewed prefill workload, alpha * ln(p_e / p_max) with
     p_e proportional to rank_e^-s over a seeded permutation of the experts;
@@ -63,6 +64,7 @@ class LayerShape:
     zipf_s: float = 0.0  # popularity exponent realised through the bias (0: none)
     zipf_alpha: float = 0.0
     seed: int = 0
+    group_size: int = 0  # 0: one weight scale per row; else one per row and group of this many codes
 
     def row_bytes(self, matrix: int) -> int:
         k = self.H if matrix in (GATE, UP) else self.I
@@ -74,9 +76,13 @@ class LayerShape:
     def matrix_bytes(self, matrix: int) -> int:
         return self.rows(matrix) * self.row_bytes(matrix)
 
+    def scales_per_row(self, matrix: int) -> int:
+        k = self.H if matrix in (GATE, UP) else self.I
+        return k // self.group_size if self.group_size else 1
+
     def expert_bytes(self) -> int:
-        """Packed codes plus fp32 per-row scales of one expert (gate, up, down)."""
-        return sum(self.matrix_bytes(m) + 4 * self.rows(m) for m in (GATE, UP, DOWN))
+        """Packed codes plus fp32 scales of one expert (gate, up, down)."""
+        return sum(self.matrix_bytes(m) + 4 * self.rows(m) * self.scales_per_row(m) for m in (GATE, UP, DOWN))
 
     def router_bytes(self) -> int:
         return 4 * self.E * self.H
@@ -252,7 +258,7 @@ def hidden_states(sh: LayerShape, layer: int = 0, tokens=None) -> np.ndarray:
 
 
 def expert_matrix(sh: LayerShape, layer: int, expert: int, matrix: int):
-    """(packed codes uint8 [rows, row_bytes], scales fp32 [rows]) of one matrix.
+    """(packed codes uint8 [rows, row_bytes], scales fp32 [rows] or, grouped, [rows, groups]) of one matrix.
 
     expert == SHARED selects the shared expert.
     """
@@ -262,8 +268,9 @@ def expert_matrix(sh: LayerShape, layer: int, expert: int, matrix: int):
         codes = codes_i8(sh.seed, sid, 0, rows * rb).view(np.uint8)
     else:
         codes = uniform_bytes(sh.seed, sid, 0, rows * rb)
-    sc = scales(sh.seed, stream_id(layer, expert, _SCALES[matrix], sh.qtype), 0, rows)
-    return codes.reshape(rows, rb), sc
+    spr = sh.scales_per_row(matrix)
+    sc = scales(sh.seed, stream_id(layer, expert, _SCALES[matrix], sh.qtype), 0, rows * spr)
+    return codes.reshape(rows, rb), (sc.reshape(rows, spr) if sh.group_size else sc)
 
 
 def fill_matrix_gpu(sh: LayerShape, layer: int, expert: int, matrix: int,
@@ -279,6 +286,6 @@ def fill_matrix_gpu(sh: LayerShape, layer: int, expert: int, matrix: int,
     if rc != 0:
         raise RuntimeError(f"synth_gpu codes launch failed: cudaError {rc}")
     rc = lib.synth_gpu_scales(sh.seed, stream_id(layer, expert, _SCALES[matrix], sh.qtype), 0,
-                              rows, SCALE_LO, SCALE_SPAN, scales_ptr, cuda_stream)
+                              rows * sh.scales_per_row(matrix), SCALE_LO, SCALE_SPAN, scales_ptr, cuda_stream)
     if rc != 0:
         raise RuntimeError(f"synth_gpu scales launch failed: cudaError {rc}")

@@ -465,6 +465,66 @@ def test_qdot_against_fp64_dequantised_dot():
         assert abs(got - ref) <= 1e-5 * scale
 
 
+@pytest.mark.parametrize("group", [32, 128])
+def test_qdot_grouped_exact_integer_case(group):
+    # every weight scale 1 and activation scales 1: the integer dot exactly
+    rng = np.random.default_rng(40 + group)
+    n = 2048
+    for _ in range(10):
+        codes = rng.integers(-8, 8, n).astype(np.int8)
+        x = rng.integers(-127, 128, n).astype(np.float32)
+        x[::32] = 127.0
+        qa, da = O.q8_0(x)
+        want = int(np.dot(codes.astype(np.int64), x.astype(np.int64)))
+        assert O.qdot_grouped(codes, np.ones(n // group, np.float32), group, qa, da) == float(want)
+
+
+@pytest.mark.parametrize("group", [32, 64, 128, 2048])
+def test_qdot_grouped_against_fp64_dequantised_dot(group):
+    # sum_k s_w[g(k)] q_w[k] d_a[b(k)] q_a[k] in fp64; each group's scale applies to its codes only
+    rng = np.random.default_rng(50 + group)
+    n = 2048
+    for _ in range(30):
+        codes = rng.integers(-8, 8, n).astype(np.int8)
+        x = rng.standard_normal(n).astype(np.float32)
+        sw = rng.uniform(0.01, 0.05, n // group).astype(np.float32)
+        qa, da = O.q8_0(x)
+        terms = (codes.astype(np.float64) * np.repeat(sw.astype(np.float64), group)
+                 * qa.astype(np.float64) * np.repeat(da.astype(np.float64), 32))
+        got = O.qdot_grouped(codes, sw, group, qa, da)
+        assert abs(got - terms.sum()) <= 1e-5 * np.abs(terms).sum()
+        if group < n:  # doubling one group's scale moves only that group's share
+            sw2 = sw.copy()
+            sw2[1] *= 2
+            d = O.qdot_grouped(codes, sw2, group, qa, da) - got
+            share = terms[group:2 * group].sum()
+            assert abs(d - share) <= 1e-5 * np.abs(terms).sum()
+
+
+@pytest.mark.parametrize("qtype,group", [(4, 32), (4, 128), (8, 64), (2, 32)])
+def test_expert_grouped_against_fp64_dense(qtype, group):
+    sh = synth.CONFIGS["tiny"].with_(qtype=qtype, H=512, I=256, group_size=group)
+    x = synth.bf16_to_f32(synth.hidden_states(sh)[0])
+    ex = oracle_experts(sh, [3])
+    y, h = O.expert_token(ex, 3, x, want_h=True)
+    g, sg = synth.expert_matrix(sh, 0, 3, synth.GATE)
+    u, su = synth.expert_matrix(sh, 0, 3, synth.UP)
+    d, sd = synth.expert_matrix(sh, 0, 3, synth.DOWN)
+    assert sg.shape == (sh.I, sh.H // group) and sd.shape == (sh.H, sh.I // group)
+    Wg = unpack_ref(g, qtype) * np.repeat(sg.astype(np.float64), group, axis=1)
+    Wu = unpack_ref(u, qtype) * np.repeat(su.astype(np.float64), group, axis=1)
+    Wd = unpack_ref(d, qtype) * np.repeat(sd.astype(np.float64), group, axis=1)
+    qa, da = O.q8_0(x)
+    xa = qa.astype(np.float64) * np.repeat(da.astype(np.float64), 32)
+    gg, uu = Wg @ xa, Wu @ xa
+    h64 = gg / (1.0 + np.exp(-gg)) * uu
+    assert np.allclose(h, h64, rtol=1e-5, atol=1e-6 * np.abs(h64).max())
+    qh, dh = O.q8_0(h.astype(np.float32))
+    ha = qh.astype(np.float64) * np.repeat(dh.astype(np.float64), 32)
+    y64, mag = Wd @ ha, np.abs(Wd) @ np.abs(ha)
+    assert np.all(np.abs(y - y64) <= 1e-5 * mag + 1e-30)
+
+
 def _round_f32(q):
     """The fp32 value nearest the rational q (ties to even), found exactly."""
     from fractions import Fraction
@@ -573,15 +633,20 @@ def test_expert_zero_gate_gives_zero_output():
 
 
 # ------------------------------------------------------ union == per-token
-@pytest.mark.parametrize("cfg", ["tiny", "verify_small"])
+@pytest.mark.parametrize("cfg", ["tiny", "verify_small", "tiny_grouped", "tiny_topp"])
 def test_union_path_equals_per_token_path_bitwise(cfg):
+    top_p = 0.0
     if cfg == "tiny":
         sh = synth.CONFIGS["tiny"]
+    elif cfg == "tiny_grouped":
+        sh = synth.CONFIGS["tiny"].with_(group_size=64)
+    elif cfg == "tiny_topp":
+        sh, top_p = synth.CONFIGS["tiny"].with_(T=12, top_k=4), 0.6
     else:
         sh = synth.CONFIGS["verify"].with_(H=512, I=256, E=32, n_group=4, topk_group=2, top_k=4, T=6)
     x, W, b = synth.hidden_states(sh), synth.router_weight(sh), synth.router_bias(sh)
-    idx, w, _, _ = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
-    ex = oracle_experts(sh, np.unique(idx))
+    idx, w, _, _ = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf, top_p=top_p)
+    ex = oracle_experts(sh, np.unique(idx[idx >= 0]))
     un = O.union(idx, sh.E)
     y_union = O.expert_ffn(ex, x, sh.top_k, un)
     y_tok = O.expert_ffn_per_token(ex, x, idx)
