@@ -100,7 +100,16 @@ typedef struct {
  *   w_down:       [n_expert][hidden][inter*qtype/8]
  *   s_gate, s_up: [n_expert][inter] fp32 row scales;  s_down: [n_expert][hidden]
  * hidden and inter must be multiples of 32 (one Q8_0 block);
- * hidden, inter <= 16384. */
+ * hidden, inter <= 16384.
+ * Grouped weight scales ([MO] "int4 양자화 (Quantization)의 품질 비용": grouped
+ * scales recover most of int4's quality loss), group_size = G != 0: one fp32
+ * scale per row and group of G consecutive codes along the row instead of one
+ * per row; G a multiple of 32 that divides hidden and inter; s_gate, s_up:
+ * [n_expert][inter][hidden/G]; s_down: [n_expert][hidden][inter/G].  Block b
+ * of a row then takes the factor d_b * s[g(b)] (rounded once to fp32) in the
+ * fold of the quantised dot and the row has no separate scale.  Batches above
+ * the fused kernel's size take the general path with grouped scales (the
+ * tensor-core path reports MOE_PATH_GENERAL for them). */
 typedef struct {
     int qtype;
     int n_expert;
@@ -112,6 +121,7 @@ typedef struct {
     const float* s_gate;
     const float* s_up;
     const float* s_down;
+    int group_size;  /* 0: per-row scales as above; else grouped scales (see below) */
 } moe_experts;
 
 /* ------------------------------------------------------------------ route */

@@ -91,6 +91,8 @@ int check_experts(const moe_experts* ex) {
     if (ex->n_expert <= 0 || ex->hidden <= 0 || ex->inter <= 0) return MOE_EINVAL;
     if (ex->hidden % 32 || ex->inter % 32) return MOE_EINVAL;
     if (ex->hidden > 16384 || ex->inter > 16384) return MOE_EUNSUPPORTED;
+    const int gs = ex->group_size;
+    if (gs < 0 || (gs && (gs % 32 || ex->hidden % gs || ex->inter % gs))) return MOE_EINVAL;
     const void* ps[6] = {ex->w_gate, ex->w_up, ex->w_down, ex->s_gate, ex->s_up, ex->s_down};
     for (const void* p : ps)
         if (!p || !aligned16(p)) return MOE_EINVAL;
@@ -182,7 +184,8 @@ bool fused_params(FusedParams& f, const LayerWs& L, void* ws, const uint16_t* x,
                   const moe_experts& r, const moe_experts* s, void* out, int out_dtype,
                   int32_t* idx, float* w) {
     if (T > kFusedMaxTokens) return false;
-    if (s && (s->qtype != r.qtype || s->inter != r.inter || s->hidden != r.hidden)) return false;
+    if (s && (s->qtype != r.qtype || s->inter != r.inter || s->hidden != r.hidden || s->group_size != r.group_size))
+        return false;
     f = FusedParams{};
     f.x = x;
     f.T = T;

@@ -267,7 +267,7 @@ __device__ __forceinline__ uint8_t* act_slot(const FusedParams& p, const Smem& s
 // Poll limit of a wait: its default, or the workspace's test limit when that
 // is set (nonzero) and smaller (see moe_workspace_set_wait_limit).
 __device__ __forceinline__ long lim(const Smem& s, long dflt) {
-    const long k = s.flag[2];
+    const long k = *reinterpret_cast<volatile const int*>(s.flag + 2);
     return k > 0 && k < dflt ? k : dflt;
 }
 
@@ -348,11 +348,12 @@ struct Segments {
 };
 
 // ------------------------------------------------------------------ producer
-template <int QT>
+template <int QT, bool G>
 __device__ void producer(const FusedParams& p, const Smem& s) {
     const size_t slot_bytes = static_cast<size_t>(p.stage_bytes) + kScaleBytes;
     const uint64_t pol = l2_evict_first_policy();
     const int nrt = p.n_rt, nug = p.n_ugt, nd = p.n_dt, hs = p.has_shared;
+    constexpr bool gs = G;  // grouped weight scales are read in place, not staged
     const int P = p.T * p.K;
     const size_t rb_ug = static_cast<size_t>(p.H) * QT / 8, rb_d = static_cast<size_t>(p.I) * QT / 8;
     int stage = 0, aslot = 0;
@@ -490,8 +491,9 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                     d.last = (m == 1 && q == kUgTileRows / kStageRows - 1);
                     d.sit = m * (kUgTileRows / kStageRows) + q;
                     const size_t r = static_cast<size_t>(d.e) * p.I + d.row0;
-                    ok = issue(d, wm + r * rb_ug, static_cast<uint32_t>(kStageRows * rb_ug), sm + r,
-                               kStageRows * 4);
+                    // per-row scales travel with the stage; grouped ones are read in place
+                    ok = issue(d, wm + r * rb_ug, static_cast<uint32_t>(kStageRows * rb_ug), gs ? nullptr : sm + r,
+                               gs ? 0u : kStageRows * 4);
                 }
             }
         } else {  // down tile: rows j*dr .. j*dr+dr-1; the helper warp copies its
@@ -521,8 +523,8 @@ __device__ void producer(const FusedParams& p, const Smem& s) {
                 d.first = q == 0;
                 d.last = q == kDownStagesPerTile - 1;
                 const size_t r = static_cast<size_t>(d.e) * p.H + d.row0;
-                ok = issue(d, ex.w_down + r * rb_d, static_cast<uint32_t>(d.nrows * rb_d), ex.s_down + r,
-                           static_cast<uint32_t>(d.nrows * 4));
+                ok = issue(d, ex.w_down + r * rb_d, static_cast<uint32_t>(d.nrows * rb_d), gs ? nullptr : ex.s_down + r,
+                           gs ? 0u : static_cast<uint32_t>(d.nrows * 4));
             }
             if (++aslot == p.nact) {
                 aslot = 0;
@@ -874,7 +876,7 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
             const int nkept = __popc(keep);
             if ((keep >> e) & 1u) {
                 const int pos = __popc(keep & ((1u << e) - 1u));
-                rs->pe[t * K + pos] = ex[e];
+                rs->pe[t * K + pos] = h.slot[e];
                 s.rt_w[t * K + pos] = __fmul_rn(__fdiv_rn(mys, den), p.rsf);
             }
             if (e >= nkept) {
@@ -955,11 +957,32 @@ struct ActRegs {
     uint4 a1[NC];
 };
 
+// Grouped weight scales ([MO] "int4 양자화 (Quantization)의 품질 비용") of row
+// `rs` of a stage, or null with per-row scales (those travel with the stage).
+// Block b's factor is then d_b * s[b / gpb] (one rounding) and the row has no
+// separate scale.
+template <bool G>
+__device__ __forceinline__ const float* grouped_row(const FusedParams& p, const Desc& d, int rs) {
+    if constexpr (!G) return nullptr;
+    const int gs = p.routed.group_size;
+    const moe_experts& ex = d.cslot == 0 ? p.shared : p.routed;  // slot 0: the shared expert
+    const size_t row = static_cast<size_t>(d.row0 + rs);
+    if (d.mat == 2) return ex.s_down + (static_cast<size_t>(d.e) * p.H + row) * (p.I / gs);
+    return (d.mat == 0 ? ex.s_gate : ex.s_up) + (static_cast<size_t>(d.e) * p.I + row) * (p.H / gs);
+}
+
+__device__ __forceinline__ float block_factor(float da, const float* sg, int b, int gpb) {
+    return sg ? __fmul_rn(da, __ldg(sg + b / gpb)) : da;
+}
+
 // up/gate stage, NT = 1: the token's Q8_0(x) words are in registers.
-template <int QT>
-__device__ __forceinline__ void consume_ug_reg(const FusedParams& p, const Smem& s, float* dst, int row0,
+template <int QT, bool G>
+__device__ __forceinline__ void consume_ug_reg(const FusedParams& p, const Smem& s, const Desc& d, float* dst,
                                                const uint8_t* sbuf, const ActRegs<kRegChunksUg>& ar, int gw) {
     const int lane = threadIdx.x & 31;
+    const int row0 = d.row0, gpb = p.routed.group_size / 32;
+    const float* sg0 = grouped_row<G>(p, d, gw);
+    const float* sg1 = grouped_row<G>(p, d, gw + kGroupWarps);
     const int nbH = p.H / 32;
     const size_t rb = static_cast<size_t>(p.H) * QT / 8;
     const uint8_t* w0 = sbuf + gw * rb;                  // rows gw and gw + kGroupWarps of the stage
@@ -973,8 +996,10 @@ __device__ __forceinline__ void consume_ug_reg(const FusedParams& p, const Smem&
             const WBlock<QT> wb1 = load_wblock_smem<QT>(w1, b);
             const int qs = s.qs[b];
             const float qd = s.qd[b];
-            acc0 = fmaf(static_cast<float>(block_dot<QT>(wb0, ar.a0[j], ar.a1[j], qs)), qd, acc0);
-            acc1 = fmaf(static_cast<float>(block_dot<QT>(wb1, ar.a0[j], ar.a1[j], qs)), qd, acc1);
+            acc0 = fmaf(static_cast<float>(block_dot<QT>(wb0, ar.a0[j], ar.a1[j], qs)), block_factor(qd, sg0, b, gpb),
+                        acc0);
+            acc1 = fmaf(static_cast<float>(block_dot<QT>(wb1, ar.a0[j], ar.a1[j], qs)), block_factor(qd, sg1, b, gpb),
+                        acc1);
         }
     }
 #pragma unroll
@@ -984,13 +1009,13 @@ __device__ __forceinline__ void consume_ug_reg(const FusedParams& p, const Smem&
     }
     if (lane == 0) {
         const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
-        dst[row0 % kUgTileRows + gw] = __fmul_rn(acc0, sc[gw]);
-        dst[row0 % kUgTileRows + gw + kGroupWarps] = __fmul_rn(acc1, sc[gw + kGroupWarps]);
+        dst[row0 % kUgTileRows + gw] = sg0 ? acc0 : __fmul_rn(acc0, sc[gw]);
+        dst[row0 % kUgTileRows + gw + kGroupWarps] = sg1 ? acc1 : __fmul_rn(acc1, sc[gw + kGroupWarps]);
     }
 }
 
 // up/gate stage, NT > 1: activations read from the shared-memory cache.
-template <int QT, int NT>
+template <int QT, int NT, bool G>
 __device__ __forceinline__ void consume_ug_smem(const FusedParams& p, const Smem& s, const Desc& d, float* dst,
                                                 const uint8_t* sbuf, int gw) {
     const int lane = threadIdx.x & 31;
@@ -1005,18 +1030,21 @@ __device__ __forceinline__ void consume_ug_smem(const FusedParams& p, const Smem
     for (int h = 0; h < 2; ++h) {  // rows gw and gw + kGroupWarps of the stage
         const int rs = gw + h * kGroupWarps;
         const uint8_t* wrow = sbuf + rs * rb;
+        const float* sg = grouped_row<G>(p, d, rs);
+        const int gpb = p.routed.group_size / 32;
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
 #pragma unroll 2
         for (int b = lane; b < nbH; b += 32) {
             const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
+            const float gsc = sg ? __ldg(sg + b / gpb) : 1.0f;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 if (t < n_tok) {
                     const int q = tok[t] * nbH + b;
                     const int isum = block_dot<QT>(wb, s.q0[q], s.q1[q], s.qs[q]);
-                    acc[t] = fmaf(static_cast<float>(isum), s.qd[q], acc[t]);
+                    acc[t] = fmaf(static_cast<float>(isum), sg ? __fmul_rn(s.qd[q], gsc) : s.qd[q], acc[t]);
                 }
             }
         }
@@ -1025,18 +1053,19 @@ __device__ __forceinline__ void consume_ug_smem(const FusedParams& p, const Smem
         for (int t = 0; t < NT; ++t) {
             if (t < n_tok) {
                 const float v = warp_sum_f32(acc[t]);
-                if (lane == 0) dst[t * kUgTileRows + r] = __fmul_rn(v, sc[rs]);
+                if (lane == 0) dst[t * kUgTileRows + r] = sg ? v : __fmul_rn(v, sc[rs]);
             }
         }
     }
 }
 
 // down stage, NT = 1: the pair's Q8_0(h) words are in registers (loaded per tile).
-template <int QT>
-__device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0, int nrows, int pair,
-                                                 const uint8_t* sbuf, const ActRegs<kRegChunksDown>& ar,
-                                                 const float* ad, const int32_t* as, int gw) {
+template <int QT, bool G>
+__device__ __forceinline__ void consume_down_reg(const FusedParams& p, const Desc& d, const uint8_t* sbuf,
+                                                 const ActRegs<kRegChunksDown>& ar, const float* ad,
+                                                 const int32_t* as, int gw) {
     const int lane = threadIdx.x & 31;
+    const int row0 = d.row0, nrows = d.nrows, pair = d.pair[0], gpb = p.routed.group_size / 32;
     const int nbI = p.I / 32;
     const size_t rb = static_cast<size_t>(p.I) * QT / 8;
     const float* sc = reinterpret_cast<const float*>(sbuf + p.stage_bytes);
@@ -1047,13 +1076,14 @@ __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0,
         const int r = gw + kGroupWarps * k;
         if (r < nrows) {
             const uint8_t* wrow = sbuf + r * rb;
+            const float* sg = grouped_row<G>(p, d, r);
 #pragma unroll
             for (int j = 0; j < kRegChunksDown; ++j) {
                 const int b = lane + 32 * j;
                 if (b < nbI) {
                     const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
                     const int isum = block_dot<QT>(wb, ar.a0[j], ar.a1[j], as[b]);
-                    acc[k] = fmaf(static_cast<float>(isum), ad[b], acc[k]);
+                    acc[k] = fmaf(static_cast<float>(isum), block_factor(ad[b], sg, b, gpb), acc[k]);
                 }
             }
         }
@@ -1063,13 +1093,13 @@ __device__ __forceinline__ void consume_down_reg(const FusedParams& p, int row0,
         const int r = gw + kGroupWarps * k;
         if (r < nrows) {
             const float v = warp_sum_f32(acc[k]);
-            if (lane == 0) p.y[static_cast<size_t>(pair) * p.H + row0 + r] = __fmul_rn(v, sc[r]);
+            if (lane == 0) p.y[static_cast<size_t>(pair) * p.H + row0 + r] = G ? v : __fmul_rn(v, sc[r]);
         }
     }
 }
 
 // down stage, NT > 1: activations read from the tile's shared-memory slot.
-template <int QT, int NT>
+template <int QT, int NT, bool G>
 __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Smem& s, const Desc& d,
                                                   const uint8_t* sbuf, int gw) {
     const int lane = threadIdx.x & 31;
@@ -1081,14 +1111,17 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
     int pair[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) pair[t] = d.pair[t];
+    const int gpb = p.routed.group_size / 32;
     for (int r = gw; r < nrows; r += kGroupWarps) {
         const uint8_t* wrow = sbuf + r * rb;
+        const float* sg = grouped_row<G>(p, d, r);
         float acc[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
 #pragma unroll 2
         for (int b = lane; b < nbI; b += 32) {
             const WBlock<QT> wb = load_wblock_smem<QT>(wrow, b);
+            const float gsc = sg ? __ldg(sg + b / gpb) : 1.0f;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 if (t < n_tok) {
@@ -1097,7 +1130,7 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
                     const uint4 a1 = reinterpret_cast<const uint4*>(rec + p.I / 2)[b];
                     const float da = reinterpret_cast<const float*>(rec + p.I)[b];
                     const int as = reinterpret_cast<const int32_t*>(rec + p.I + nbI * 4)[b];
-                    acc[t] = fmaf(static_cast<float>(block_dot<QT>(wb, a0, a1, as)), da, acc[t]);
+                    acc[t] = fmaf(static_cast<float>(block_dot<QT>(wb, a0, a1, as)), sg ? __fmul_rn(da, gsc) : da, acc[t]);
                 }
             }
         }
@@ -1105,7 +1138,7 @@ __device__ __forceinline__ void consume_down_smem(const FusedParams& p, const Sm
         for (int t = 0; t < NT; ++t) {
             if (t < n_tok) {
                 const float v = warp_sum_f32(acc[t]);
-                if (lane == 0) p.y[static_cast<size_t>(pair[t]) * p.H + row0 + r] = __fmul_rn(v, sc[r]);
+                if (lane == 0) p.y[static_cast<size_t>(pair[t]) * p.H + row0 + r] = sg ? v : __fmul_rn(v, sc[r]);
             }
         }
     }
@@ -1131,7 +1164,7 @@ __device__ __forceinline__ void push_task(const Smem& s, int tb, const Desc* d, 
     if (lane == 0) mbar_arrive(&s.tfull[tb]);
 }
 
-template <int QT, int NT>
+template <int QT, int NT, bool G>
 __device__ void consumer(const FusedParams& p, const Smem& s) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = warp / kGroupWarps, gw = warp % kGroupWarps;
@@ -1211,9 +1244,9 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                 }
                 float* dst = (d.mat == 0 ? s.gbuf : s.ubuf) + tb * kMaxT * kUgTileRows;
                 if constexpr (NT == 1) {
-                    consume_ug_reg<QT>(p, s, dst, d.row0, sbuf, ar, gw);
+                    consume_ug_reg<QT, G>(p, s, d, dst, sbuf, ar, gw);
                 } else {
-                    consume_ug_smem<QT, NT>(p, s, d, dst, sbuf, gw);
+                    consume_ug_smem<QT, NT, G>(p, s, d, dst, sbuf, gw);
                 }
                 if (d.sit + kGroups >= d.nst) {
                     push_task(s, tb, &d, D_UG, d.sit == d.nst - 1 && gw == 0);
@@ -1250,9 +1283,9 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
                     }
                 }
                 if constexpr (NT == 1) {
-                    consume_down_reg<QT>(p, d.row0, d.nrows, d.pair[0], sbuf, ar, ad, as, gw);
+                    consume_down_reg<QT, G>(p, d, sbuf, ar, ad, as, gw);
                 } else {
-                    consume_down_smem<QT, NT>(p, s, d, sbuf, gw);
+                    consume_down_smem<QT, NT, G>(p, s, d, sbuf, gw);
                 }
                 if (d.sit + kGroups >= d.nst) {
                     __syncwarp();
@@ -1288,6 +1321,9 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
 template <int QT>
 __device__ __forceinline__ void helper_warp(const FusedParams& p, const Smem& s) {
     if ((threadIdx.x & 31) != 0) return;
+    // the workspace's test limit on bounded waits, off every other warp's start-up path
+    // (written by the host before the launch; waits use their defaults until it lands)
+    atomicExch(&s.flag[2], ld_relaxed_gpu(&p.sync->wait_limit));
     long n_act = 0;
     int slot = 0;
     uint32_t ph = 0;
@@ -1369,23 +1405,29 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
                 // every load of an element first (they are L2 round trips, at
                 // the end of the launch), then the sum in slot order
                 const int c0 = blk * p.dr, nr = min(p.dr, p.H - c0), K = p.K;
-                for (int i = lane; i < p.T * nr; i += 32) {
-                    const int t = i / nr, c = c0 + i % nr;
-                    // an empty slot (weight 0, no pair) adds nothing
-                    float yv[kMaxExpertsPerLane];
+                for (int t = 0; t < p.T; ++t) {
+                    // the token's slots, once: an empty slot (weight 0, no pair) adds nothing
+                    float wk[kMaxExpertsPerLane];
+                    const float* yk[kMaxExpertsPerLane];
 #pragma unroll
-                    for (int k = 0; k < kMaxExpertsPerLane; ++k)
-                        yv[k] = k < K && s.rt_w[t * K + k] != 0.0f
-                                    ? __ldcg(p.y + static_cast<size_t>(s.rt_pair_of[t * K + k]) * p.H + c)
-                                    : 0.0f;
-                    float o = p.has_shared ? __ldcg(p.y + static_cast<size_t>(P + t) * p.H + c) : 0.0f;
+                    for (int k = 0; k < kMaxExpertsPerLane; ++k) {
+                        wk[k] = k < K ? s.rt_w[t * K + k] : 0.0f;
+                        yk[k] = wk[k] != 0.0f ? p.y + static_cast<size_t>(s.rt_pair_of[t * K + k]) * p.H : nullptr;
+                    }
+                    for (int i = lane; i < nr; i += 32) {
+                        const int c = c0 + i;
+                        float yv[kMaxExpertsPerLane];
 #pragma unroll
-                    for (int k = 0; k < kMaxExpertsPerLane; ++k)
-                        if (k < K && s.rt_w[t * K + k] != 0.0f) o = __fadd_rn(o, __fmul_rn(s.rt_w[t * K + k], yv[k]));
-                    if (p.out_bf16) {
-                        static_cast<uint16_t*>(p.out)[static_cast<size_t>(t) * p.H + c] = f32_to_bf16_bits(o);
-                    } else {
-                        static_cast<float*>(p.out)[static_cast<size_t>(t) * p.H + c] = o;
+                        for (int k = 0; k < kMaxExpertsPerLane; ++k) yv[k] = yk[k] ? __ldcg(yk[k] + c) : 0.0f;
+                        float o = p.has_shared ? __ldcg(p.y + static_cast<size_t>(P + t) * p.H + c) : 0.0f;
+#pragma unroll
+                        for (int k = 0; k < kMaxExpertsPerLane; ++k)
+                            if (yk[k]) o = __fadd_rn(o, __fmul_rn(wk[k], yv[k]));
+                        if (p.out_bf16) {
+                            static_cast<uint16_t*>(p.out)[static_cast<size_t>(t) * p.H + c] = f32_to_bf16_bits(o);
+                        } else {
+                            static_cast<float*>(p.out)[static_cast<size_t>(t) * p.H + c] = o;
+                        }
                     }
                 }
             }
@@ -1396,7 +1438,7 @@ __device__ void epilogue_warp(const FusedParams& p, const Smem& s, int tb) {
     }
 }
 
-template <int QT, int NT>
+template <int QT, int NT, bool G>
 __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_constant__ FusedParams p) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     const Smem s = carve(smem_raw, p);
@@ -1424,7 +1466,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfree[i], 1);
         }
         mbar_init(s.route_bar, 1);
-        s.flag[2] = ld_relaxed_gpu(&p.sync->wait_limit);  // set by the host before the launch
+        s.flag[2] = 0;  // the test limit on waits: the helper warp fetches it (default until then)
         for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.areq_full[i], 1);
             mbar_init(&s.areq_free[i], 1);
@@ -1441,13 +1483,13 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
         named_bar_sync(kBarAfterDep, kThreadsF - 32);
     }
     if (warp == kProducerWarp) {
-        if (lane == 0) producer<QT>(p, s);
+        if (lane == 0) producer<QT, G>(p, s);
     } else if (warp == kHelperWarp) {
         helper_warp<QT>(p, s);
     } else if (warp >= kEpilogueWarp0) {
         epilogue_warp<QT>(p, s, warp - kEpilogueWarp0);
     } else {
-        consumer<QT, NT>(p, s);
+        consumer<QT, NT, G>(p, s);
     }
     __syncthreads();
     if (tid == 0) {
@@ -1465,9 +1507,12 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
 }
 
 template <int QT>
-const void* fused_kernel(int nt) {
-    return nt == 1 ? reinterpret_cast<const void*>(k_decode_fused<QT, 1>)
-                   : reinterpret_cast<const void*>(k_decode_fused<QT, kMaxT>);
+const void* fused_kernel(int nt, bool grouped) {
+    if (grouped)
+        return nt == 1 ? reinterpret_cast<const void*>(k_decode_fused<QT, 1, true>)
+                       : reinterpret_cast<const void*>(k_decode_fused<QT, kMaxT, true>);
+    return nt == 1 ? reinterpret_cast<const void*>(k_decode_fused<QT, 1, false>)
+                   : reinterpret_cast<const void*>(k_decode_fused<QT, kMaxT, false>);
 }
 
 }  // namespace
@@ -1522,9 +1567,9 @@ cudaError_t launch_decode_fused(const FusedParams& p, cudaStream_t st) {
     const size_t smem = fused_smem_bytes(p);
     const void* kern;
     switch (p.routed.qtype) {
-        case MOE_Q_INT4: kern = fused_kernel<4>(p.nt); break;
-        case MOE_Q_INT8: kern = fused_kernel<8>(p.nt); break;
-        case MOE_Q_INT2: kern = fused_kernel<2>(p.nt); break;
+        case MOE_Q_INT4: kern = fused_kernel<4>(p.nt, p.routed.group_size != 0); break;
+        case MOE_Q_INT8: kern = fused_kernel<8>(p.nt, p.routed.group_size != 0); break;
+        case MOE_Q_INT2: kern = fused_kernel<2>(p.nt, p.routed.group_size != 0); break;
         default: return cudaErrorInvalidValue;
     }
     e = ensure_smem(kern, smem);

@@ -8,7 +8,9 @@
 // Every weight row is consumed by one lane, which folds the row's 32-code
 // blocks in ascending order with one fp32 fused multiply-add per block: the
 // quantised dot of the layer's definition, bit for bit (a one-ulp difference in
-// h could flip a Q8_0 code of h).
+// h could flip a Q8_0 code of h).  With grouped weight scales ([MO] "int4
+// 양자화 (Quantization)의 품질 비용") block b's factor is d_b * s[g(b)], rounded
+// once, and the row has no separate scale.
 //
 // up/gate kernel: one CTA per (32-row block of h, distinct expert).  It stages
 // the Q8_0 activations of up to kUgTok of the expert's tokens in shared
@@ -54,21 +56,24 @@ __device__ __forceinline__ bool expert_range(const UnionView& un, int u, int T, 
 
 // Lane-per-row quantised dots of one weight row against TPW staged activation
 // rows (t0 .. t0 + nt - 1 of the staging area): blocks ascending, one fused
-// multiply-add per block; returns the unscaled sums.
+// multiply-add per block; returns the sums before any per-row scale.  sg: the
+// row's grouped scales (gpb blocks per group), or null for per-row scales.
 template <int QT, int TPW>
 __device__ __forceinline__ void row_dots(const uint8_t* row, int nb, const uint4* a0, const uint4* a1,
                                          const float* ad, const int32_t* as, int t0, int nt,
-                                         float (&acc)[TPW]) {
+                                         const float* sg, int gpb, float (&acc)[TPW]) {
 #pragma unroll
     for (int t = 0; t < TPW; ++t) acc[t] = 0.0f;
 #pragma unroll 4
     for (int b = 0; b < nb; ++b) {
         const WBlock<QT> w = load_wblock_l1<QT>(row, b);
+        const float gw = sg ? __ldg(sg + b / gpb) : 1.0f;
 #pragma unroll
         for (int t = 0; t < TPW; ++t) {
             if (t < nt) {
                 const int q = (t0 + t) * nb + b;
-                acc[t] = fmaf(static_cast<float>(block_dot<QT>(w, a0[q], a1[q], as[q])), ad[q], acc[t]);
+                const float f = sg ? __fmul_rn(ad[q], gw) : ad[q];
+                acc[t] = fmaf(static_cast<float>(block_dot<QT>(w, a0[q], a1[q], as[q])), f, acc[t]);
             }
         }
     }
@@ -77,7 +82,7 @@ __device__ __forceinline__ void row_dots(const uint8_t* row, int nb, const uint4
 template <int QT>
 __global__ void __launch_bounds__(kThreads)
 k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
-          const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I,
+          const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I, int gs,
           const int8_t* __restrict__ qx, const float* __restrict__ dx, int T, UnionView un,
           int8_t* __restrict__ qh, float* __restrict__ dh) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -97,7 +102,9 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     const int m = warp & 1, tg = warp >> 1;  // gate / up rows; token group
     const size_t row = static_cast<size_t>(er.e) * I + r0 + lane;
     const uint8_t* wrow = (m == 0 ? w_gate : w_up) + row * rb;
-    const float srow = __ldg((m == 0 ? s_gate : s_up) + row);
+    const float* sbase = m == 0 ? s_gate : s_up;
+    const float* sg = gs ? sbase + row * (H / gs) : nullptr;  // grouped: the row's scales
+    const float srow = gs ? 1.0f : __ldg(sbase + row);
     float* dst = m == 0 ? gbuf : ubuf;
 
     for (int pc = er.p0; pc < er.p1; pc += kUgTok) {
@@ -112,10 +119,10 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
         const int t0 = tg * kUgTpw, ntw = min(kUgTpw, nt - t0);
         if (ntw > 0) {
             float acc[kUgTpw];
-            row_dots<QT, kUgTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, acc);
+            row_dots<QT, kUgTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, sg, gs / 32, acc);
 #pragma unroll
             for (int t = 0; t < kUgTpw; ++t)
-                if (t < ntw) dst[(t0 + t) * kUgRows + lane] = __fmul_rn(acc[t], srow);
+                if (t < ntw) dst[(t0 + t) * kUgRows + lane] = gs ? acc[t] : __fmul_rn(acc[t], srow);
         }
         __syncthreads();
         for (int t = warp; t < nt; t += kWarps) {
@@ -132,7 +139,7 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
 
 template <int QT>
 __global__ void __launch_bounds__(kThreads)
-k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I,
+k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I, int gs,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
        float* __restrict__ y_pairs) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -149,7 +156,8 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t row = static_cast<size_t>(er.e) * H + c0 + lane;
     const uint8_t* wrow = w_down + row * rb;
-    const float srow = __ldg(s_down + row);
+    const float* sg = gs ? s_down + row * (I / gs) : nullptr;  // grouped: the row's scales
+    const float srow = gs ? 1.0f : __ldg(s_down + row);
 
     for (int pc = er.p0; pc < er.p1; pc += kDownTok) {
         const int nt = min(kDownTok, er.p1 - pc);
@@ -162,14 +170,14 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
         const int t0 = warp * kDownTpw, ntw = min(kDownTpw, nt - t0);
         if (ntw > 0) {
             float acc[kDownTpw];
-            row_dots<QT, kDownTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, acc);
+            row_dots<QT, kDownTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, sg, gs / 32, acc);
 #pragma unroll
             for (int t = 0; t < kDownTpw; ++t) {
                 if (t < ntw) {
                     const int p = pc + t0 + t;
                     const int tok = un.uniq ? un.pair_tok[p] : p;
                     const int slot = un.uniq ? un.pair_slot[p] : 0;
-                    y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + lane] = __fmul_rn(acc[t], srow);
+                    y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + lane] = gs ? acc[t] : __fmul_rn(acc[t], srow);
                 }
             }
         }
@@ -187,7 +195,7 @@ cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx,
     if (e != cudaSuccess) return e;
     const dim3 grid(ex.inter / kUgRows, un.max_unique);
     kern<<<grid, kThreads, smem, st>>>(ex.w_gate, ex.w_up, ex.s_gate, ex.s_up, ex.hidden, ex.inter,
-                                       qx, dx, T, un, qh, dh);
+                                       ex.group_size, qx, dx, T, un, qh, dh);
     return counted(cudaGetLastError());
 }
 
@@ -200,7 +208,8 @@ cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, in
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const dim3 grid(ex.hidden / kDownRows, un.max_unique);
-    kern<<<grid, kThreads, smem, st>>>(ex.w_down, ex.s_down, ex.hidden, ex.inter, qh, dh, T, K, un, y);
+    kern<<<grid, kThreads, smem, st>>>(ex.w_down, ex.s_down, ex.hidden, ex.inter, ex.group_size, qh, dh, T, K,
+                                       un, y);
     return counted(cudaGetLastError());
 }
 

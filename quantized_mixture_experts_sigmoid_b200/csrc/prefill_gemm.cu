@@ -603,6 +603,7 @@ size_t gemm_smem_bytes() {
 bool tc_gemm_supported(const moe_experts& r, const moe_experts* s, int E) {
     if (r.qtype != MOE_Q_INT4 || (s && (s->qtype != MOE_Q_INT4 || s->inter != r.inter || s->hidden != r.hidden)))
         return false;
+    if (r.group_size || (s && s->group_size)) return false;  // per-row scales only (the epilogue's fold)
     if (r.hidden % kBK || r.inter % kBK) return false;  // whole K stages; 64-column output halves
     if (E + 1 > kMaxItems) return false;
     return true;

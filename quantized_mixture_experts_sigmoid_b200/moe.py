@@ -45,7 +45,7 @@ class _Experts(ctypes.Structure):
     _fields_ = [("qtype", ctypes.c_int), ("n_expert", ctypes.c_int), ("hidden", ctypes.c_int),
                 ("inter", ctypes.c_int), ("w_gate", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
                 ("w_down", ctypes.c_void_p), ("s_gate", ctypes.c_void_p),
-                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p)]
+                ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p), ("group_size", ctypes.c_int)]
 
 
 @dataclass
@@ -53,7 +53,8 @@ class ExpertSet:
     """A stack of experts resident on the device (tensors owned by the caller).
 
     w_gate, w_up: uint8 [n, inter, hidden*q/8]; w_down: uint8 [n, hidden, inter*q/8];
-    s_gate, s_up: fp32 [n, inter]; s_down: fp32 [n, hidden].
+    s_gate, s_up: fp32 [n, inter]; s_down: fp32 [n, hidden]; with grouped scales (group_size G)
+    s_gate, s_up: fp32 [n, inter, hidden/G]; s_down: fp32 [n, hidden, inter/G].
     """
     qtype: int
     n_expert: int
@@ -65,22 +66,25 @@ class ExpertSet:
     s_gate: torch.Tensor
     s_up: torch.Tensor
     s_down: torch.Tensor
+    group_size: int = 0
 
     def struct(self) -> _Experts:
         return _Experts(self.qtype, self.n_expert, self.hidden, self.inter, self.w_gate.data_ptr(),
                         self.w_up.data_ptr(), self.w_down.data_ptr(), self.s_gate.data_ptr(),
-                        self.s_up.data_ptr(), self.s_down.data_ptr())
+                        self.s_up.data_ptr(), self.s_down.data_ptr(), self.group_size)
 
     @staticmethod
-    def empty(qtype: int, n_expert: int, hidden: int, inter: int, device="cuda") -> "ExpertSet":
+    def empty(qtype: int, n_expert: int, hidden: int, inter: int, device="cuda", group_size: int = 0) -> "ExpertSet":
         u8 = dict(dtype=torch.uint8, device=device)
         f32 = dict(dtype=torch.float32, device=device)
+        gh = (hidden // group_size,) if group_size else ()
+        gi = (inter // group_size,) if group_size else ()
         return ExpertSet(qtype, n_expert, hidden, inter,
                          torch.empty(n_expert, inter, hidden * qtype // 8, **u8),
                          torch.empty(n_expert, inter, hidden * qtype // 8, **u8),
                          torch.empty(n_expert, hidden, inter * qtype // 8, **u8),
-                         torch.empty(n_expert, inter, **f32), torch.empty(n_expert, inter, **f32),
-                         torch.empty(n_expert, hidden, **f32))
+                         torch.empty(n_expert, inter, *gh, **f32), torch.empty(n_expert, inter, *gh, **f32),
+                         torch.empty(n_expert, hidden, *gi, **f32), group_size)
 
 
 _lib = None

@@ -29,11 +29,11 @@ def device_layer(sh: synth.LayerShape, layer: int = 0, routed: moe.ExpertSet | N
                  with_shared: bool = True):
     """routed + shared ExpertSets, router weight and bias on the device, router cfg."""
     if routed is None:
-        routed = moe.ExpertSet.empty(sh.qtype, sh.E, sh.H, sh.I)
+        routed = moe.ExpertSet.empty(sh.qtype, sh.E, sh.H, sh.I, group_size=sh.group_size)
     fill_experts(sh, layer, range(sh.E), routed)
     shared = None
     if with_shared:
-        shared = moe.ExpertSet.empty(sh.qtype, 1, sh.H, sh.I)
+        shared = moe.ExpertSet.empty(sh.qtype, 1, sh.H, sh.I, group_size=sh.group_size)
         fill_experts(sh, layer, [synth.SHARED], shared, slot_of=lambda e: 0)
     W = torch.from_numpy(synth.router_weight(sh, layer)).cuda()
     b = torch.from_numpy(synth.router_bias(sh, layer)).cuda()

@@ -44,8 +44,8 @@ def _cfg(E=256, G=8, TG=4, K=8, rsf=2.5):
     return moe.RouterCfg(E, G, TG, K, rsf)
 
 
-def _ex(q=4, n=256, H=6144, I=2048, ptr=P):
-    return moe._Experts(q, n, H, I, ptr, ptr, ptr, ptr, ptr, ptr)
+def _ex(q=4, n=256, H=6144, I=2048, ptr=P, group=0):
+    return moe._Experts(q, n, H, I, ptr, ptr, ptr, ptr, ptr, ptr, group)
 
 
 @pytest.mark.parametrize("cfg", [_cfg(E=0), _cfg(G=3), _cfg(G=64, E=64), _cfg(TG=9), _cfg(K=0),
@@ -156,3 +156,18 @@ def test_usage_calls_reject_bad_arguments_without_a_gpu():
     assert L.moe_usage_accumulate(P, 0, 8, 256, P, None) == moe.MOE_OK  # empty batch: nothing to add
     assert L.moe_usage_rank(P, 0, P, None) == moe.MOE_EINVAL
     assert L.moe_usage_rank(None, 256, P, None) == moe.MOE_EINVAL
+
+
+def test_grouped_scales_geometry_and_paths_on_the_host():
+    # group sizes: a multiple of 32 dividing hidden and inter; the fused kernel takes
+    # grouped scales, the tensor-core GEMMs do not (those batches report the general path)
+    L = moe.lib()
+    c = _cfg()
+    path = lambda T, r, s: L.moe_layer_path(T, ctypes.byref(c), ctypes.byref(r), ctypes.byref(s))
+    assert path(1, _ex(group=48), _ex(n=1, group=48)) == moe.MOE_EINVAL
+    assert path(1, _ex(group=96), _ex(n=1, group=96)) == moe.MOE_EINVAL  # 2048 % 96 != 0
+    assert path(1, _ex(group=-32), _ex(n=1, group=-32)) == moe.MOE_EINVAL
+    assert path(1, _ex(group=128), _ex(n=1, group=128)) == moe.PATH_FUSED
+    assert path(40, _ex(group=128), _ex(n=1, group=128)) == moe.PATH_GENERAL
+    assert path(40, _ex(), _ex(n=1)) == moe.PATH_TENSOR_CORE
+    assert path(1, _ex(group=128), _ex(n=1, group=32)) == moe.PATH_GENERAL  # mixed sizes: not fused
