@@ -89,7 +89,6 @@ constexpr long kEpilogueWait = 1L << 25;
 // (The drains that wait for this CTA's own copies in flight keep kProducerWait
 // whatever the test limit below says: a copy may not land after the exit.)
 constexpr int kBarConsumers = 1;     // named barrier id of the consumer warps (group g: 2 + g)
-constexpr int kBarAfterDep = 4;      // all warps but the producer, after the grid dependency
 static_assert(kStageRows == 2 * kGroupWarps, "an up/gate stage gives each warp of a group two rows");
 static_assert(kDownStagesPerTile == kGroups && (2 * (kUgTileRows / kStageRows)) % kGroups == 0,
               "the stages of every tile reach every consumer group");
@@ -1466,6 +1465,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
             mbar_init(&s.tfree[i], 1);
         }
         mbar_init(s.route_bar, 1);
+        *s.rt_U = -1;  // until the routing sets it
         s.flag[2] = 0;  // the test limit on waits: the helper warp fetches it (default until then)
         for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.areq_full[i], 1);
@@ -1476,11 +1476,12 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
     }
     __syncthreads();
     // everyone but the producer waits for the previous grid here (x, the
-    // workspace and its launch counter may come from it)
+    // workspace and its launch counter may come from it).  Only the consumers
+    // read this launch's tag, after the barrier that ends consumer_init, so
+    // its load overlaps theirs of x.
     if (warp != kProducerWarp) {
         grid_dependency_wait();
         if (tid == 0) *s.tag = static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch))) + 1u;
-        named_bar_sync(kBarAfterDep, kThreadsF - 32);
     }
     if (warp == kProducerWarp) {
         if (lane == 0) producer<QT, G>(p, s);
@@ -1491,17 +1492,25 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
     } else {
         consumer<QT, NT, G>(p, s);
     }
+    // Count this CTA out: the add releases the counters its warps advanced
+    // (ordered before it by the barrier) and, in the last CTA, acquires every
+    // other CTA's.  The last CTA then clears what this launch advanced for the
+    // next call on this workspace: completion counters 0 .. U (the shared
+    // expert and the U routed ones; all of them if the routing did not finish)
+    // and the row-block counters.  Kernel completion makes the stores visible
+    // to the next grid.
     __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        if (atomicAdd(&p.sync->exit_count, 1) == static_cast<int>(gridDim.x) - 1) {
-            // last CTA out: reset the counters for the next call on this workspace
-            for (int i = 0; i <= p.E; ++i) p.ug_done[i] = 0;
-            for (int i = 0; i < p.n_dt; ++i) p.rb_done[i] = 0;
+    if (tid == 0) s.flag[0] = atom_add_acq_rel_gpu(&p.sync->exit_count, 1) == static_cast<int>(gridDim.x) - 1;
+    __syncthreads();
+    if (s.flag[0]) {
+        const int nu = *s.rt_U;
+        const int nr = nu >= 0 && nu < p.E ? nu : p.E;
+        for (int i = tid; i <= nr; i += kThreadsF) p.ug_done[i] = 0;
+        for (int i = tid; i < p.n_dt; i += kThreadsF) p.rb_done[i] = 0;
+        if (tid == 0) {
             p.sync->ticket = 0;
             p.sync->exit_count = 0;
             *p.epoch = *s.tag;
-            __threadfence();
         }
     }
 }
