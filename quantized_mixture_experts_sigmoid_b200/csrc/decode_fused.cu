@@ -576,18 +576,17 @@ __device__ __forceinline__ void store_q8_block_warp(float v, uint32_t* w_lo, uin
 }
 
 // ------------------------------------------------------------------ consumers
-// Q8_0 of every token's x (all consumer threads; TPB threads per 32-block),
+// Q8_0 of every token's x (threads idx of nth; TPB threads per 32-block),
 // stored permuted for dp4a against qtype QT.  Same arithmetic as q8_0_lane.
 // Each thread's permuted words hold only its own elements, so no exchange
 // through shared memory is needed: thread `part` of a block owns elements
 // [part EPT, part EPT + EPT) and words [part WPT, part WPT + WPT).
 template <int QT>
-__device__ __forceinline__ void quantize_x(const FusedParams& p, const Smem& s) {
+__device__ __forceinline__ void quantize_x(const FusedParams& p, const Smem& s, int idx, int nth) {
     constexpr int TPB = QT == 2 ? 2 : 4, EPT = 32 / TPB, WPT = 8 / TPB;
-    const int tid = threadIdx.x;
     const int nbH = p.H / 32, ntask = p.T * nbH * TPB;
-    for (int base = 0; base < ntask; base += kConsumers) {
-        const int task = base + tid;
+    for (int base = 0; base < ntask; base += nth) {
+        const int task = base + idx;
         const bool active = task < ntask;
         const int blk = task / TPB, part = task % TPB;
         float v[EPT];
@@ -613,12 +612,23 @@ __device__ __forceinline__ void quantize_x(const FusedParams& p, const Smem& s) 
 #pragma unroll
         for (int o = 1; o < TPB; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float d = __fdiv_rn(amax, 127.0f);
+        // q = round(v / d) with the correctly rounded quotient.  t = v * RN(1/d)
+        // is within 2.5e-5 of RN(v / d) while |v / d| <= 127, so where t lies
+        // farther than 1e-4 from a half-integer both round to the same
+        // integer; elsewhere (and when 1/d overflows) the division decides.
+        const float r = d != 0.0f ? __frcp_rn(d) : 0.0f;
         int q[EPT];
         int sum = 0;
 #pragma unroll
         for (int i = 0; i < EPT; ++i) {
-            int qi = 0;
-            if (d != 0.0f) qi = static_cast<int>(fminf(fmaxf(roundf(__fdiv_rn(v[i], d)), -127.0f), 127.0f));
+            const float t = __fmul_rn(v[i], r), a = fabsf(t);
+            float qf;
+            if (a <= 128.0f && fabsf(a - floorf(a) - 0.5f) >= 1e-4f) {
+                qf = roundf(t);
+            } else {
+                qf = roundf(__fdiv_rn(v[i], d));
+            }
+            const int qi = d != 0.0f ? static_cast<int>(fminf(fmaxf(qf, -127.0f), 127.0f)) : 0;
             q[i] = qi;
             sum += qi;
         }
@@ -647,12 +657,16 @@ __device__ __forceinline__ void quantize_x(const FusedParams& p, const Smem& s) 
     }
 }
 
+// x and the bias into shared memory, and this launch's tag (the previous
+// launch's number + 1), whose load overlaps those of x.
 __device__ void consumer_init(const FusedParams& p, const Smem& s) {
     const int tid = threadIdx.x;
+    const int ep = tid == 0 ? ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch)) : 0;
     const int n16 = p.T * p.H / 8;
     for (int i = tid; i < n16; i += kConsumers)
         reinterpret_cast<uint4*>(s.xs)[i] = reinterpret_cast<const uint4*>(p.x)[i];
     for (int e = tid; e < p.E; e += kConsumers) s.bias[e] = __ldg(p.bias + e);
+    if (tid == 0) *s.tag = static_cast<uint32_t>(ep) + 1u;
     consumers_sync();
 }
 
@@ -1202,8 +1216,15 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
         tph[tb] ^= 1u;
         tb ^= 1;
     };
+    // phase A: the router rows up to the route marker, Q8_0 of x, then the
+    // routing.  A CTA's router rows start at its stage 0 (group 0); for one
+    // token, when the last group's first stage holds none, that group
+    // quantises x meanwhile.
     int type = next_type();
-    // phase A: router rows up to the route marker, Q8_0 of x, then the routing
+    if (p.T == 1 && g == kGroups - 1 && type != D_ROUTER) {
+        quantize_x<QT>(p, s, tid % kGroupThreads, kGroupThreads);
+        if (tid % kGroupThreads == 0) s.flag[1] = 1;
+    }
     while (type == D_ROUTER) {
         const int e0 = s.desc[stage].e, nrows = s.desc[stage].nrows;
         consume_router<NT>(p, s, e0, nrows, s.ring + stage * slot_bytes, g);
@@ -1212,8 +1233,11 @@ __device__ void consumer(const FusedParams& p, const Smem& s) {
     }
     const bool marker = type == D_MARK;
     if (marker) release();
-    quantize_x<QT>(p, s);
     consumers_sync();
+    if (s.flag[1] == 0) {  // the last group had router rows: everyone quantises x now
+        quantize_x<QT>(p, s, tid, kConsumers);
+        consumers_sync();
+    }
     route_block(p, s);  // the x cache holds the routing scratch from here on
     if (marker) type = next_type();
     // phases B and C: runs of up/gate tiles and of down tiles.  A tile's
@@ -1466,6 +1490,7 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
         }
         mbar_init(s.route_bar, 1);
         *s.rt_U = -1;  // until the routing sets it
+        s.flag[1] = 0;  // set once x is quantised during the router rows
         s.flag[2] = 0;  // the test limit on waits: the helper warp fetches it (default until then)
         for (int i = 0; i < kMaxActSlots; ++i) {
             mbar_init(&s.areq_full[i], 1);
@@ -1476,13 +1501,8 @@ __global__ void __launch_bounds__(kThreadsF, 1) k_decode_fused(const __grid_cons
     }
     __syncthreads();
     // everyone but the producer waits for the previous grid here (x, the
-    // workspace and its launch counter may come from it).  Only the consumers
-    // read this launch's tag, after the barrier that ends consumer_init, so
-    // its load overlaps theirs of x.
-    if (warp != kProducerWarp) {
-        grid_dependency_wait();
-        if (tid == 0) *s.tag = static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int*>(p.epoch))) + 1u;
-    }
+    // workspace and its launch counter may come from it)
+    if (warp != kProducerWarp) grid_dependency_wait();
     if (warp == kProducerWarp) {
         if (lane == 0) producer<QT, G>(p, s);
     } else if (warp == kHelperWarp) {
