@@ -836,9 +836,13 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
             int rank = 0;
             for (uint32_t km = kept; km; km &= km - 1) {
                 const ulonglong2* c2 = reinterpret_cast<const ulonglong2*>(h.cand + (__ffs(km) - 1) * gsz);
-                for (int i = 0; i < gsz / 2; ++i) {
-                    const ulonglong2 v = c2[i];
-                    rank += (v.x > mine) + (v.y > mine);
+                // 32 experts a warp: the group's loads all issued before the compares
+                for (int i0 = 0; i0 < gsz / 2; i0 += 16) {
+                    ulonglong2 v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = c2[i0 + i];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) rank += (v[i].x > mine) + (v[i].y > mine);
                 }
             }
             if (rank < K) h.slot[rank] = e;
@@ -917,7 +921,8 @@ __device__ void route_block(const FusedParams& p, const Smem& s) {
         // one token: distinct experts, the kept ones first; a pair's position is its expert's rank
         const uint32_t valid = __ballot_sync(all, act);
         int pos = 0;
-        for (int k = 0; k < K; ++k) pos += ((valid >> k) & 1u) && rs->pe[k] < pe;
+#pragma unroll
+        for (int k = 0; k < kMaxExpertsPerLane; ++k) pos += k < K && ((valid >> k) & 1u) && rs->pe[k] < pe;
         if (act) {
             s.rt_ptok[pos] = 0;
             s.rt_pair_of[lane] = pos;
