@@ -61,14 +61,18 @@ k_router_logits(const uint16_t* __restrict__ x, const float* __restrict__ w, int
 // shared memory in chunks of 16 along H, converted to fp64 once (double
 // buffered).  Every logit is accumulated by one thread in ascending h, the
 // order of the plain definition, so the fp64 sum is that of the definition.
+// The W chunk is stored with each thread's expert pairs side by side across
+// threads ([pair][thread][2]), so a warp's 16-byte loads of it are contiguous.
 constexpr int kTiledMinT = 32;
 constexpr int kTM = 64, kTN = 64, kKC = 16, kTiledThreads = 256;
+static_assert(kTM == 64 && kTN == 64 && kTiledThreads == 256 && kKC % 4 == 0,
+              "thread (ty, tx) = (tid / 16, tid % 16) owns tokens 4 ty.. and experts 4 tx..; the loader covers 64 rows");
 
 __global__ void __launch_bounds__(kTiledThreads)
 k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ w, int T, int H, int E,
                       float* __restrict__ logits) {
     __shared__ __align__(16) double xs[2][kKC][kTM];  // [stage][h][token]
-    __shared__ __align__(16) double wsm[2][kKC][kTN]; // [stage][h][expert]
+    __shared__ __align__(16) double wsm[2][kKC][kTN]; // [stage][h][expert pair half][thread][2]
     const int tid = threadIdx.x;
     const int t0 = blockIdx.x * kTM, e0 = blockIdx.y * kTN;
     const int ty = tid >> 4, tx = tid & 15;  // tokens 4 ty .. 4 ty + 3, experts 4 tx .. 4 tx + 3
@@ -92,10 +96,11 @@ k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ 
         xs[st][lc + 1][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.x >> 16)));
         xs[st][lc + 2][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.y)));
         xs[st][lc + 3][lr] = static_cast<double>(bf16_bits_to_f32(static_cast<uint16_t>(xr.y >> 16)));
-        wsm[st][lc + 0][lr] = static_cast<double>(wr.x);
-        wsm[st][lc + 1][lr] = static_cast<double>(wr.y);
-        wsm[st][lc + 2][lr] = static_cast<double>(wr.z);
-        wsm[st][lc + 3][lr] = static_cast<double>(wr.w);
+        const int wc = ((lr & 3) >> 1) * (kTN / 2) + (lr >> 2) * 2 + (lr & 1);  // expert lr of the tile
+        wsm[st][lc + 0][wc] = static_cast<double>(wr.x);
+        wsm[st][lc + 1][wc] = static_cast<double>(wr.y);
+        wsm[st][lc + 2][wc] = static_cast<double>(wr.z);
+        wsm[st][lc + 3][wc] = static_cast<double>(wr.w);
         __syncthreads();
         if (kc + 1 < nk) {  // the next chunk's values, in flight during this chunk's products
             xr = xin ? __ldg(reinterpret_cast<const uint2*>(xrow + (kc + 1) * kKC)) : make_uint2(0, 0);
@@ -105,8 +110,8 @@ k_router_logits_tiled(const uint16_t* __restrict__ x, const float* __restrict__ 
         for (int k = 0; k < kKC; ++k) {
             const double2 a01 = *reinterpret_cast<const double2*>(&xs[st][k][4 * ty]);
             const double2 a23 = *reinterpret_cast<const double2*>(&xs[st][k][4 * ty + 2]);
-            const double2 b01 = *reinterpret_cast<const double2*>(&wsm[st][k][4 * tx]);
-            const double2 b23 = *reinterpret_cast<const double2*>(&wsm[st][k][4 * tx + 2]);
+            const double2 b01 = *reinterpret_cast<const double2*>(&wsm[st][k][2 * tx]);
+            const double2 b23 = *reinterpret_cast<const double2*>(&wsm[st][k][kTN / 2 + 2 * tx]);
             const double a[4] = {a01.x, a01.y, a23.x, a23.y}, bb[4] = {b01.x, b01.y, b23.x, b23.y};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
