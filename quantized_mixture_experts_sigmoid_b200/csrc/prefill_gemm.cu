@@ -63,7 +63,7 @@ constexpr int kWarpProducer = 0, kWarpMma = 1, kWarpXform0 = 2, kXformWarps = 4,
 // the host); warpgroups 0-1 (producer, MMA, dequantisers) lower their limit to
 // kRegsLow and the epilogue warpgroups 2-3 raise theirs to kRegsHigh, which
 // uses exactly the launched total: 2 x kRegsLow + 2 x kRegsHigh = 4 x kLaunchRegs.
-constexpr int kLaunchRegs = 128, kRegsLow = 32, kRegsHigh = 224;
+constexpr int kLaunchRegs = 128, kRegsLow = 48, kRegsHigh = 208;
 static_assert(2 * kRegsLow + 2 * kRegsHigh == 4 * kLaunchRegs, "register split must use the launched total");
 static_assert(kWarpEpi0 == 8 && kEpiWarps == 8, "epilogue = warpgroups 2 and 3");
 constexpr long kGemmWait = 1L << 26;            // polls of the final drain waits
