@@ -312,9 +312,9 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
  *   MOE_PATH_FUSED        one persistent launch for the whole layer (T <= 4,
  *                         T*top_k <= 32, n_expert <= 256 and a multiple of 32,
  *                         groups of a multiple of 32 experts, fits shared memory);
- *   MOE_PATH_TENSOR_CORE  batch-union FFN on tcgen05 tensor cores (T > 4, int4,
- *                         hidden and inter multiples of 64, shared expert shaped
- *                         like the routed ones);
+ *   MOE_PATH_TENSOR_CORE  batch-union FFN on tcgen05 tensor cores (T > 32, int4
+ *                         with per-row scales, hidden and inter multiples of 64,
+ *                         shared expert shaped like the routed ones);
  *   MOE_PATH_GENERAL      router, union, Q8_0, integer-dot expert kernels, combine.
  * Returns one of those or MOE_EINVAL.
  */

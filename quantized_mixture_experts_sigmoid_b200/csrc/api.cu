@@ -126,7 +126,7 @@ struct LayerWs {
     float* dhs;
     float* y;
     float* ys;
-    // tensor-core batch-union path (T > kFusedMaxTokens, int4)
+    // tensor-core batch-union path (T > kGeneralMaxTokens, int4)
     __half* xg;    // Q8_0(x) codes as fp16 per up/gate row [(P + T)][H] (union order, shared rows last)
     __half* hc;    // Q8_0(h) codes as fp16 [(P + T)][I]
     float* hs;     // their block scales
@@ -162,7 +162,7 @@ LayerWs carve_layer(void* ws, int T, const moe_router_cfg& c, const moe_experts&
         L.ys = cv.take<float>(static_cast<size_t>(T) * H);
     }
     L.y = cv.take<float>(P * H);
-    if (T > kFusedMaxTokens && tc_gemm_supported(r, s, c.n_expert)) {
+    if (T > kGeneralMaxTokens && tc_gemm_supported(r, s, c.n_expert)) {
         const size_t rows = P + static_cast<size_t>(T);
         L.xg = cv.take<__half>(rows * H);
         L.hc = cv.take<__half>(rows * I);
@@ -518,7 +518,7 @@ int moe_layer_path(int T, const moe_router_cfg* cfg, const moe_experts* routed, 
     if (fused_params(f, L, fake, fx, T, reinterpret_cast<const float*>(fake), reinterpret_cast<const float*>(fake),
                      *cfg, *routed, shared, fake, MOE_OUT_F32, nullptr, nullptr))
         return MOE_PATH_FUSED;
-    if (T > kFusedMaxTokens && tc_gemm_supported(*routed, shared, cfg->n_expert)) return MOE_PATH_TENSOR_CORE;
+    if (T > kGeneralMaxTokens && tc_gemm_supported(*routed, shared, cfg->n_expert)) return MOE_PATH_TENSOR_CORE;
     return MOE_PATH_GENERAL;
 }
 

@@ -132,7 +132,9 @@ def test_layer_path_query():
                                                           ctypes.byref(ss) if ss is not None else None)
     assert path(1) == moe.PATH_FUSED
     assert path(4) == moe.PATH_FUSED
-    assert path(5) == moe.PATH_TENSOR_CORE
+    assert path(5) == moe.PATH_GENERAL        # a few tokens per expert: lane-per-row kernels
+    assert path(32) == moe.PATH_GENERAL
+    assert path(33) == moe.PATH_TENSOR_CORE
     assert path(2048) == moe.PATH_TENSOR_CORE
     assert path(2048, rr=_ex(q=8)) == moe.PATH_GENERAL           # int8 experts: integer-dot kernels
     assert path(2048, rr=_ex(H=544, I=288), ss=_ex(n=1, H=544, I=288)) == moe.PATH_GENERAL  # K not a multiple of 64
