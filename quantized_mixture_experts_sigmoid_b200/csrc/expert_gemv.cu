@@ -8,7 +8,10 @@
 // Every weight row is consumed by one lane, which folds the row's 32-code
 // blocks in ascending order with one fp32 fused multiply-add per block: the
 // quantised dot of the layer's definition, bit for bit (a one-ulp difference in
-// h could flip a Q8_0 code of h).  With grouped weight scales ([MO] "int4
+// h could flip a Q8_0 code of h).  The CTA's weight rows pass through shared
+// memory in chunks of kCB blocks, loaded with coalesced 16-byte (int2: 8-byte)
+// reads one chunk ahead in registers: a lane streaming its own row through L1
+// would need more L1 than the SM has beside the staging buffers.  With grouped weight scales ([MO] "int4
 // 양자화 (Quantization)의 품질 비용") block b's factor is d_b * s[g(b)], rounded
 // once, and the row has no separate scale.
 //
@@ -20,6 +23,8 @@
 // down kernel: one CTA per (32 output rows, distinct expert); warp w takes
 // kDownTpw of the expert's staged pairs, lane r output row r; y is written by
 // (token, slot).
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "quant.cuh"
@@ -35,6 +40,61 @@ constexpr int kUgTpw = 2;                       // tokens per warp (up/gate)
 constexpr int kUgTok = kUgTpw * kWarps / 2;     // tokens staged per pass (up/gate): 8
 constexpr int kDownTpw = 2;                     // pairs per warp (down)
 constexpr int kDownTok = kDownTpw * kWarps;     // pairs staged per pass (down): 16
+
+constexpr int kCB = 32;  // weight blocks of a row per staged chunk
+
+// Chunk c (blocks c kCB .. c kCB + kCB - 1) of NR weight rows, staged through
+// registers into shared memory rows of kStride bytes.  Thread tid takes pieces
+// tid, tid + kThreads, ... in row-major order, so a warp reads contiguous bytes
+// of a row.  Pieces past the end of a row (a last, partial chunk) read nothing.
+template <int QT, int NR>
+struct WeightChunk {
+    static constexpr int kPiece = QT == 2 ? 8 : 16;           // one int2 block, or 16 bytes
+    static constexpr int kChunkBytes = kCB * 4 * QT;           // a row's bytes per chunk
+    static constexpr int kStride = kChunkBytes + kPiece;       // padded: conflict-free lane-per-row reads
+    static constexpr int kPieces = kChunkBytes / kPiece;       // pieces per row per chunk
+    static constexpr int kPerThread = NR * kPieces / kThreads;
+    static constexpr int kBytes = NR * kStride;                // shared memory
+    static_assert(NR * kPieces % kThreads == 0, "whole pieces per thread");
+    using Piece = typename std::conditional<QT == 2, uint2, uint4>::type;
+    Piece v[kPerThread];
+
+    template <class RowPtr>
+    __device__ __forceinline__ void load(const RowPtr& row_ptr, size_t row_bytes, int c) {
+#pragma unroll
+        for (int j = 0; j < kPerThread; ++j) {
+            const int u = j * kThreads + static_cast<int>(threadIdx.x);
+            const int r = u / kPieces, pc = u % kPieces;
+            const size_t off = static_cast<size_t>(c) * kChunkBytes + static_cast<size_t>(pc) * kPiece;
+            v[j] = off < row_bytes ? __ldg(reinterpret_cast<const Piece*>(row_ptr(r) + off)) : Piece{};
+        }
+    }
+    __device__ __forceinline__ void store(uint8_t* dst) const {
+#pragma unroll
+        for (int j = 0; j < kPerThread; ++j) {
+            const int u = j * kThreads + static_cast<int>(threadIdx.x);
+            const int r = u / kPieces, pc = u % kPieces;
+            *reinterpret_cast<Piece*>(dst + r * kStride + pc * kPiece) = v[j];
+        }
+    }
+};
+
+template <int QT>
+__device__ __forceinline__ WBlock<QT> wblock_staged(const uint8_t* row, int i) {
+    WBlock<QT> r;
+    if constexpr (QT == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(row + 8 * i);
+        r.w[0] = v.x;
+        r.w[1] = v.y;
+    } else {
+#pragma unroll
+        for (int h = 0; h < QT / 4; ++h) {
+            const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * (QT / 4 * i + h));
+            r.w[4 * h] = v.x; r.w[4 * h + 1] = v.y; r.w[4 * h + 2] = v.z; r.w[4 * h + 3] = v.w;
+        }
+    }
+    return r;
+}
 
 struct ExpertRange {
     int e, p0, p1;
@@ -55,18 +115,18 @@ __device__ __forceinline__ bool expert_range(const UnionView& un, int u, int T, 
 }
 
 // Lane-per-row quantised dots of one weight row against TPW staged activation
-// rows (t0 .. t0 + nt - 1 of the staging area): blocks ascending, one fused
-// multiply-add per block; returns the sums before any per-row scale.  sg: the
-// row's grouped scales (gpb blocks per group), or null for per-row scales.
+// rows (t0 .. t0 + nt - 1 of the staging area), blocks b0 .. b0 + nbc - 1 of
+// the row (its staged chunk `row`): blocks ascending, one fused multiply-add
+// per block, accumulated into acc (the sums before any per-row scale).  sg:
+// the row's grouped scales (gpb blocks per group), or null for per-row scales.
 template <int QT, int TPW>
-__device__ __forceinline__ void row_dots(const uint8_t* row, int nb, const uint4* a0, const uint4* a1,
-                                         const float* ad, const int32_t* as, int t0, int nt,
-                                         const float* sg, int gpb, float (&acc)[TPW]) {
-#pragma unroll
-    for (int t = 0; t < TPW; ++t) acc[t] = 0.0f;
+__device__ __forceinline__ void row_dots_chunk(const uint8_t* row, int b0, int nbc, int nb, const uint4* a0,
+                                               const uint4* a1, const float* ad, const int32_t* as, int t0,
+                                               int nt, const float* sg, int gpb, float (&acc)[TPW]) {
 #pragma unroll 4
-    for (int b = 0; b < nb; ++b) {
-        const WBlock<QT> w = load_wblock_l1<QT>(row, b);
+    for (int i = 0; i < nbc; ++i) {
+        const int b = b0 + i;
+        const WBlock<QT> w = wblock_staged<QT>(row, i);
         const float gw = sg ? __ldg(sg + b / gpb) : 1.0f;
 #pragma unroll
         for (int t = 0; t < TPW; ++t) {
@@ -85,9 +145,11 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
           const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I, int gs,
           const int8_t* __restrict__ qx, const float* __restrict__ dx, int T, UnionView un,
           int8_t* __restrict__ qh, float* __restrict__ dh) {
+    using Chunk = WeightChunk<QT, 2 * kUgRows>;  // the CTA's 32 gate rows, then its 32 up rows
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = H / 32;
-    uint4* a0 = reinterpret_cast<uint4*>(smem);
+    uint8_t* wsm = smem;
+    uint4* a0 = reinterpret_cast<uint4*>(smem + Chunk::kBytes);
     uint4* a1 = a0 + kUgTok * nb;
     float* ad = reinterpret_cast<float*>(a1 + kUgTok * nb);
     int32_t* as = reinterpret_cast<int32_t*>(ad + kUgTok * nb);
@@ -101,7 +163,11 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m = warp & 1, tg = warp >> 1;  // gate / up rows; token group
     const size_t row = static_cast<size_t>(er.e) * I + r0 + lane;
-    const uint8_t* wrow = (m == 0 ? w_gate : w_up) + row * rb;
+    const uint8_t* gate0 = w_gate + (static_cast<size_t>(er.e) * I + r0) * rb;
+    const uint8_t* up0 = w_up + (static_cast<size_t>(er.e) * I + r0) * rb;
+    const auto row_ptr = [&](int r) { return r < kUgRows ? gate0 + r * rb : up0 + (r - kUgRows) * rb; };
+    const uint8_t* wrow = wsm + (m * kUgRows + lane) * Chunk::kStride;
+    const int nchunks = (nb + kCB - 1) / kCB;
     const float* sbase = m == 0 ? s_gate : s_up;
     const float* sg = gs ? sbase + row * (H / gs) : nullptr;  // grouped: the row's scales
     const float srow = gs ? 1.0f : __ldg(sbase + row);
@@ -115,11 +181,22 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
                               nb, a0 + i * nb, a1 + i * nb, ad + i * nb, as + i * nb, threadIdx.x,
                               kThreads);
         }
-        __syncthreads();
         const int t0 = tg * kUgTpw, ntw = min(kUgTpw, nt - t0);
+        float acc[kUgTpw];
+#pragma unroll
+        for (int t = 0; t < kUgTpw; ++t) acc[t] = 0.0f;
+        Chunk wc;
+        wc.load(row_ptr, rb, 0);
+        for (int c = 0; c < nchunks; ++c) {
+            __syncthreads();  // activations staged; the previous chunk consumed
+            wc.store(wsm);
+            __syncthreads();
+            if (c + 1 < nchunks) wc.load(row_ptr, rb, c + 1);  // in flight while this chunk is used
+            if (ntw > 0)
+                row_dots_chunk<QT, kUgTpw>(wrow, c * kCB, min(kCB, nb - c * kCB), nb, a0, a1, ad, as, t0, ntw,
+                                           sg, gs / 32, acc);
+        }
         if (ntw > 0) {
-            float acc[kUgTpw];
-            row_dots<QT, kUgTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, sg, gs / 32, acc);
 #pragma unroll
             for (int t = 0; t < kUgTpw; ++t)
                 if (t < ntw) dst[(t0 + t) * kUgRows + lane] = gs ? acc[t] : __fmul_rn(acc[t], srow);
@@ -142,9 +219,11 @@ __global__ void __launch_bounds__(kThreads)
 k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I, int gs,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
        float* __restrict__ y_pairs) {
+    using Chunk = WeightChunk<QT, kDownRows>;
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = I / 32;
-    uint4* a0 = reinterpret_cast<uint4*>(smem);
+    uint8_t* wsm = smem;
+    uint4* a0 = reinterpret_cast<uint4*>(smem + Chunk::kBytes);
     uint4* a1 = a0 + kDownTok * nb;
     float* ad = reinterpret_cast<float*>(a1 + kDownTok * nb);
     int32_t* as = reinterpret_cast<int32_t*>(ad + kDownTok * nb);
@@ -155,7 +234,10 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
     const size_t rb = static_cast<size_t>(I) * QT / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const size_t row = static_cast<size_t>(er.e) * H + c0 + lane;
-    const uint8_t* wrow = w_down + row * rb;
+    const uint8_t* down0 = w_down + (static_cast<size_t>(er.e) * H + c0) * rb;
+    const auto row_ptr = [&](int r) { return down0 + r * rb; };
+    const uint8_t* wrow = wsm + lane * Chunk::kStride;
+    const int nchunks = (nb + kCB - 1) / kCB;
     const float* sg = gs ? s_down + row * (I / gs) : nullptr;  // grouped: the row's scales
     const float srow = gs ? 1.0f : __ldg(s_down + row);
 
@@ -166,11 +248,22 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
             stage_act_row<QT>(qh + p * I, dh + p * nb, nb, a0 + i * nb, a1 + i * nb, ad + i * nb,
                               as + i * nb, threadIdx.x, kThreads);
         }
-        __syncthreads();
         const int t0 = warp * kDownTpw, ntw = min(kDownTpw, nt - t0);
+        float acc[kDownTpw];
+#pragma unroll
+        for (int t = 0; t < kDownTpw; ++t) acc[t] = 0.0f;
+        Chunk wc;
+        wc.load(row_ptr, rb, 0);
+        for (int c = 0; c < nchunks; ++c) {
+            __syncthreads();  // activations staged; the previous chunk consumed
+            wc.store(wsm);
+            __syncthreads();
+            if (c + 1 < nchunks) wc.load(row_ptr, rb, c + 1);
+            if (ntw > 0)
+                row_dots_chunk<QT, kDownTpw>(wrow, c * kCB, min(kCB, nb - c * kCB), nb, a0, a1, ad, as, t0, ntw,
+                                             sg, gs / 32, acc);
+        }
         if (ntw > 0) {
-            float acc[kDownTpw];
-            row_dots<QT, kDownTpw>(wrow, nb, a0, a1, ad, as, t0, ntw, sg, gs / 32, acc);
 #pragma unroll
             for (int t = 0; t < kDownTpw; ++t) {
                 if (t < ntw) {
@@ -189,7 +282,8 @@ template <int QT>
 cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
                        const UnionView& un, int8_t* qh, float* dh, cudaStream_t st) {
     const int nb = ex.hidden / 32;
-    const size_t smem = static_cast<size_t>(kUgTok) * nb * 40 + 2 * kUgTok * kUgRows * sizeof(float);
+    const size_t smem = WeightChunk<QT, 2 * kUgRows>::kBytes + static_cast<size_t>(kUgTok) * nb * 40 +
+                        2 * kUgTok * kUgRows * sizeof(float);
     auto kern = k_up_gate<QT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
@@ -203,7 +297,7 @@ template <int QT>
 cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, int T, int K,
                     const UnionView& un, float* y, cudaStream_t st) {
     const int nb = ex.inter / 32;
-    const size_t smem = static_cast<size_t>(kDownTok) * nb * 40;
+    const size_t smem = WeightChunk<QT, kDownRows>::kBytes + static_cast<size_t>(kDownTok) * nb * 40;
     auto kern = k_down<QT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
