@@ -35,7 +35,7 @@ k_router_logits(const uint16_t* __restrict__ x, const float* __restrict__ w, int
     for (int t = 0; t < TT; ++t) acc[t] = 0.0;
     const float4* w4 = reinterpret_cast<const float4*>(w + static_cast<size_t>(e) * H);
     const int n4 = H >> 2;
-#pragma unroll 2
+#pragma unroll 8  // eight 16-byte loads of the row in flight per lane
     for (int j = lane; j < n4; j += 32) {
         const float4 wv = __ldg(w4 + j);
 #pragma unroll
