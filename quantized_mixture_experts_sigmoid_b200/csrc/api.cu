@@ -352,9 +352,10 @@ int moe_expert_ffn_q(const moe_experts* ex, const uint16_t* x, int T, int top_k,
                  dense ? 1 : static_cast<int>(std::min<long long>(ex->n_expert, static_cast<long long>(T) * top_k))};
     rc = cuda_rc(launch_q8_0(x, true, T, ex->hidden, F.qx, F.dx, st));
     if (rc) return rc;
-    rc = cuda_rc(launch_expert_up_gate(*ex, F.qx, F.dx, T, un, F.qh, F.dh, st));
+    const int tpe = tokens_per_expert(un, T, top_k);
+    rc = cuda_rc(launch_expert_up_gate(*ex, F.qx, F.dx, T, un, tpe, F.qh, F.dh, st));
     if (rc) return rc;
-    return cuda_rc(launch_expert_down(*ex, F.qh, F.dh, T, top_k, un, y_pairs, st));
+    return cuda_rc(launch_expert_down(*ex, F.qh, F.dh, T, top_k, un, tpe, y_pairs, st));
 }
 
 int moe_combine(const float* y_pairs, const float* topk_w, const float* shared_y, int T, int top_k,
@@ -496,14 +497,15 @@ int moe_layer_forward(const uint16_t* x, int T, const float* w_router, const flo
     const UnionView un{L.n_unique, L.uniq, L.offsets, L.pair_tok, L.pair_slot,
                        static_cast<int>(std::min<long long>(E, static_cast<long long>(T) * K))};
     const bool timed = g_prof.begin(st);
-    rc = cuda_rc(launch_expert_up_gate(*routed, L.qx, L.dx, T, un, L.qh, L.dh, st));
+    const int tpe = tokens_per_expert(un, T, K);
+    rc = cuda_rc(launch_expert_up_gate(*routed, L.qx, L.dx, T, un, tpe, L.qh, L.dh, st));
     if (timed) g_prof.end(st);
     if (rc) return rc;
     const UnionView dense{nullptr, nullptr, nullptr, nullptr, nullptr, 1};
-    if (shared && (rc = cuda_rc(launch_expert_up_gate(*shared, L.qx, L.dx, T, dense, L.qhs, L.dhs, st))))
+    if (shared && (rc = cuda_rc(launch_expert_up_gate(*shared, L.qx, L.dx, T, dense, T, L.qhs, L.dhs, st))))
         return rc;
-    if ((rc = cuda_rc(launch_expert_down(*routed, L.qh, L.dh, T, K, un, L.y, st)))) return rc;
-    if (shared && (rc = cuda_rc(launch_expert_down(*shared, L.qhs, L.dhs, T, 1, dense, L.ys, st))))
+    if ((rc = cuda_rc(launch_expert_down(*routed, L.qh, L.dh, T, K, un, tpe, L.y, st)))) return rc;
+    if (shared && (rc = cuda_rc(launch_expert_down(*shared, L.qhs, L.dhs, T, 1, dense, T, L.ys, st))))
         return rc;
     return cuda_rc(launch_combine(L.y, w, shared ? L.ys : nullptr, T, K, H, out, out_dtype, st));
 }

@@ -34,28 +34,43 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUgRows = 32;                     // h rows per up/gate CTA
-constexpr int kDownRows = 32;                   // output rows per down CTA
-constexpr int kUgTpw = 2;                       // tokens per warp (up/gate)
-constexpr int kUgTok = kUgTpw * kWarps / 2;     // tokens staged per pass (up/gate): 8
-constexpr int kDownTpw = 2;                     // pairs per warp (down)
-constexpr int kDownTok = kDownTpw * kWarps;     // pairs staged per pass (down): 16
+constexpr int kTpw = 2;  // tokens (pairs) per warp and pass
 
-constexpr int kCB = 32;  // weight blocks of a row per staged chunk
+// CTA geometry.  Narrow: the 8 warps split into 4 token groups of 2 (up/gate:
+// 32 h rows; down: 8 groups over 32 output rows), for experts that see many
+// tokens.  Wide: every warp takes its own 32 rows (up/gate: 128 h rows; down:
+// 256 output rows) and the CTA two tokens a pass, for batches whose experts
+// see one or two tokens each: then no warp idles while the others compute.
+template <bool W>
+struct UgGeom {
+    static constexpr int kRq = W ? 4 : 1;              // 32-row groups of h per CTA
+    static constexpr int kTg = 4 / kRq;                // token groups
+    static constexpr int kRows = 32 * kRq;             // h rows per CTA
+    static constexpr int kTok = kTg * kTpw;            // tokens staged per pass
+};
+template <bool W>
+struct DownGeom {
+    static constexpr int kRd = W ? 8 : 1;              // 32-row groups of output per CTA
+    static constexpr int kPg = kWarps / kRd;           // pair groups
+    static constexpr int kRows = 32 * kRd;             // output rows per CTA
+    static constexpr int kTok = kPg * kTpw;            // pairs staged per pass
+};
 
-// Chunk c (blocks c kCB .. c kCB + kCB - 1) of NR weight rows, staged through
-// registers into shared memory rows of kStride bytes.  Thread tid takes pieces
-// tid, tid + kThreads, ... in row-major order, so a warp reads contiguous bytes
-// of a row.  Pieces past the end of a row (a last, partial chunk) read nothing.
-template <int QT, int NR>
+// Chunk c of NR weight rows (a row's bytes kBytesPerRow per chunk: kChunkBlocks
+// blocks), staged through registers into shared memory rows of kStride bytes.
+// Thread tid takes pieces tid, tid + kThreads, ... in row-major order, so a
+// warp reads contiguous bytes of a row.  Pieces past the end of a row (a last,
+// partial chunk) read nothing.
+template <int QT, int NR, int kBytesPerRow>
 struct WeightChunk {
     static constexpr int kPiece = QT == 2 ? 8 : 16;           // one int2 block, or 16 bytes
-    static constexpr int kChunkBytes = kCB * 4 * QT;           // a row's bytes per chunk
+    static constexpr int kChunkBytes = kBytesPerRow;
+    static constexpr int kChunkBlocks = kChunkBytes / (4 * QT);
     static constexpr int kStride = kChunkBytes + kPiece;       // padded: conflict-free lane-per-row reads
     static constexpr int kPieces = kChunkBytes / kPiece;       // pieces per row per chunk
     static constexpr int kPerThread = NR * kPieces / kThreads;
     static constexpr int kBytes = NR * kStride;                // shared memory
-    static_assert(NR * kPieces % kThreads == 0, "whole pieces per thread");
+    static_assert(NR * kPieces % kThreads == 0 && kChunkBytes % (4 * QT) == 0, "whole pieces and blocks");
     using Piece = typename std::conditional<QT == 2, uint2, uint4>::type;
     Piece v[kPerThread];
 
@@ -78,6 +93,10 @@ struct WeightChunk {
         }
     }
 };
+// Narrow CTAs stage 32 blocks of a row per chunk; wide ones (four or eight
+// times the rows) 256 bytes of a row.
+template <int QT, int NR, bool W>
+using ChunkOf = WeightChunk<QT, NR, W ? 256 : 32 * 4 * QT>;
 
 template <int QT>
 __device__ __forceinline__ WBlock<QT> wblock_staged(const uint8_t* row, int i) {
@@ -139,52 +158,54 @@ __device__ __forceinline__ void row_dots_chunk(const uint8_t* row, int b0, int n
     }
 }
 
-template <int QT>
+template <int QT, bool W>
 __global__ void __launch_bounds__(kThreads)
 k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
           const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I, int gs,
           const int8_t* __restrict__ qx, const float* __restrict__ dx, int T, UnionView un,
           int8_t* __restrict__ qh, float* __restrict__ dh) {
-    using Chunk = WeightChunk<QT, 2 * kUgRows>;  // the CTA's 32 gate rows, then its 32 up rows
+    using Geo = UgGeom<W>;
+    using Chunk = ChunkOf<QT, 2 * Geo::kRows, W>;  // the CTA's gate rows, then its up rows
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = H / 32;
     uint8_t* wsm = smem;
     uint4* a0 = reinterpret_cast<uint4*>(smem + Chunk::kBytes);
-    uint4* a1 = a0 + kUgTok * nb;
-    float* ad = reinterpret_cast<float*>(a1 + kUgTok * nb);
-    int32_t* as = reinterpret_cast<int32_t*>(ad + kUgTok * nb);
-    float* gbuf = reinterpret_cast<float*>(as + kUgTok * nb);
-    float* ubuf = gbuf + kUgTok * kUgRows;
+    uint4* a1 = a0 + Geo::kTok * nb;
+    float* ad = reinterpret_cast<float*>(a1 + Geo::kTok * nb);
+    int32_t* as = reinterpret_cast<int32_t*>(ad + Geo::kTok * nb);
+    float* gbuf = reinterpret_cast<float*>(as + Geo::kTok * nb);
+    float* ubuf = gbuf + Geo::kTok * Geo::kRows;
 
     ExpertRange er;
     if (!expert_range(un, blockIdx.y, T, er)) return;
-    const int r0 = blockIdx.x * kUgRows;
+    const int r0 = blockIdx.x * Geo::kRows;
     const size_t rb = static_cast<size_t>(H) * QT / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m = warp & 1, tg = warp >> 1;  // gate / up rows; token group
-    const size_t row = static_cast<size_t>(er.e) * I + r0 + lane;
+    const int m = warp & 1, g = warp >> 1, rq = g % Geo::kRq, tg = g / Geo::kRq;  // gate / up; rows; tokens
+    const int hr = rq * 32 + lane;  // this lane's h row within the CTA
+    const size_t row = static_cast<size_t>(er.e) * I + r0 + hr;
     const uint8_t* gate0 = w_gate + (static_cast<size_t>(er.e) * I + r0) * rb;
     const uint8_t* up0 = w_up + (static_cast<size_t>(er.e) * I + r0) * rb;
-    const auto row_ptr = [&](int r) { return r < kUgRows ? gate0 + r * rb : up0 + (r - kUgRows) * rb; };
-    const uint8_t* wrow = wsm + (m * kUgRows + lane) * Chunk::kStride;
-    const int nchunks = (nb + kCB - 1) / kCB;
+    const auto row_ptr = [&](int r) { return r < Geo::kRows ? gate0 + r * rb : up0 + (r - Geo::kRows) * rb; };
+    const uint8_t* wrow = wsm + (m * Geo::kRows + hr) * Chunk::kStride;
+    const int nchunks = (nb + Chunk::kChunkBlocks - 1) / Chunk::kChunkBlocks;
     const float* sbase = m == 0 ? s_gate : s_up;
     const float* sg = gs ? sbase + row * (H / gs) : nullptr;  // grouped: the row's scales
     const float srow = gs ? 1.0f : __ldg(sbase + row);
     float* dst = m == 0 ? gbuf : ubuf;
 
-    for (int pc = er.p0; pc < er.p1; pc += kUgTok) {
-        const int nt = min(kUgTok, er.p1 - pc);
+    for (int pc = er.p0; pc < er.p1; pc += Geo::kTok) {
+        const int nt = min(Geo::kTok, er.p1 - pc);
         for (int i = 0; i < nt; ++i) {
             const int tok = un.uniq ? un.pair_tok[pc + i] : pc + i;
             stage_act_row<QT>(qx + static_cast<size_t>(tok) * H, dx + static_cast<size_t>(tok) * nb,
                               nb, a0 + i * nb, a1 + i * nb, ad + i * nb, as + i * nb, threadIdx.x,
                               kThreads);
         }
-        const int t0 = tg * kUgTpw, ntw = min(kUgTpw, nt - t0);
-        float acc[kUgTpw];
+        const int t0 = tg * kTpw, ntw = min(kTpw, nt - t0);
+        float acc[kTpw];
 #pragma unroll
-        for (int t = 0; t < kUgTpw; ++t) acc[t] = 0.0f;
+        for (int t = 0; t < kTpw; ++t) acc[t] = 0.0f;
         Chunk wc;
         wc.load(row_ptr, rb, 0);
         for (int c = 0; c < nchunks; ++c) {
@@ -192,66 +213,72 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
             wc.store(wsm);
             __syncthreads();
             if (c + 1 < nchunks) wc.load(row_ptr, rb, c + 1);  // in flight while this chunk is used
+            const int b0 = c * Chunk::kChunkBlocks;
             if (ntw > 0)
-                row_dots_chunk<QT, kUgTpw>(wrow, c * kCB, min(kCB, nb - c * kCB), nb, a0, a1, ad, as, t0, ntw,
-                                           sg, gs / 32, acc);
+                row_dots_chunk<QT, kTpw>(wrow, b0, min(Chunk::kChunkBlocks, nb - b0), nb, a0, a1, ad, as, t0, ntw,
+                                         sg, gs / 32, acc);
         }
         if (ntw > 0) {
 #pragma unroll
-            for (int t = 0; t < kUgTpw; ++t)
-                if (t < ntw) dst[(t0 + t) * kUgRows + lane] = gs ? acc[t] : __fmul_rn(acc[t], srow);
+            for (int t = 0; t < kTpw; ++t)
+                if (t < ntw) dst[(t0 + t) * Geo::kRows + hr] = gs ? acc[t] : __fmul_rn(acc[t], srow);
         }
         __syncthreads();
-        for (int t = warp; t < nt; t += kWarps) {
-            const float h = swiglu(gbuf[t * kUgRows + lane], ubuf[t * kUgRows + lane]);
+        // SwiGLU and Q8_0 of each token's 32-row groups of h (one warp a group)
+        for (int i = warp; i < nt * Geo::kRq; i += kWarps) {
+            const int t = i / Geo::kRq, q = i % Geo::kRq;
+            const float h = swiglu(gbuf[t * Geo::kRows + q * 32 + lane], ubuf[t * Geo::kRows + q * 32 + lane]);
             float db;
-            const int8_t q = q8_0_lane(h, &db);
+            const int8_t qv = q8_0_lane(h, &db);
             const size_t p = static_cast<size_t>(pc + t);
-            qh[p * I + r0 + lane] = q;
-            if (lane == 0) dh[p * (I / 32) + blockIdx.x] = db;
+            qh[p * I + r0 + q * 32 + lane] = qv;
+            if (lane == 0) dh[p * (I / 32) + r0 / 32 + q] = db;
         }
         __syncthreads();
     }
 }
 
-template <int QT>
+template <int QT, bool W>
 __global__ void __launch_bounds__(kThreads)
 k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I, int gs,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
        float* __restrict__ y_pairs) {
-    using Chunk = WeightChunk<QT, kDownRows>;
+    using Geo = DownGeom<W>;
+    using Chunk = ChunkOf<QT, Geo::kRows, W>;
     extern __shared__ __align__(16) uint8_t smem[];
     const int nb = I / 32;
     uint8_t* wsm = smem;
     uint4* a0 = reinterpret_cast<uint4*>(smem + Chunk::kBytes);
-    uint4* a1 = a0 + kDownTok * nb;
-    float* ad = reinterpret_cast<float*>(a1 + kDownTok * nb);
-    int32_t* as = reinterpret_cast<int32_t*>(ad + kDownTok * nb);
+    uint4* a1 = a0 + Geo::kTok * nb;
+    float* ad = reinterpret_cast<float*>(a1 + Geo::kTok * nb);
+    int32_t* as = reinterpret_cast<int32_t*>(ad + Geo::kTok * nb);
 
     ExpertRange er;
     if (!expert_range(un, blockIdx.y, T, er)) return;
-    const int c0 = blockIdx.x * kDownRows;
+    const int c0 = blockIdx.x * Geo::kRows;
     const size_t rb = static_cast<size_t>(I) * QT / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const size_t row = static_cast<size_t>(er.e) * H + c0 + lane;
+    const int rg = warp % Geo::kRd, pg = warp / Geo::kRd;  // rows; pairs
+    const int orow = rg * 32 + lane;  // this lane's output row within the CTA
+    const size_t row = static_cast<size_t>(er.e) * H + c0 + orow;
     const uint8_t* down0 = w_down + (static_cast<size_t>(er.e) * H + c0) * rb;
     const auto row_ptr = [&](int r) { return down0 + r * rb; };
-    const uint8_t* wrow = wsm + lane * Chunk::kStride;
-    const int nchunks = (nb + kCB - 1) / kCB;
+    const uint8_t* wrow = wsm + orow * Chunk::kStride;
+    const int nchunks = (nb + Chunk::kChunkBlocks - 1) / Chunk::kChunkBlocks;
     const float* sg = gs ? s_down + row * (I / gs) : nullptr;  // grouped: the row's scales
     const float srow = gs ? 1.0f : __ldg(s_down + row);
 
-    for (int pc = er.p0; pc < er.p1; pc += kDownTok) {
-        const int nt = min(kDownTok, er.p1 - pc);
+    for (int pc = er.p0; pc < er.p1; pc += Geo::kTok) {
+        const int nt = min(Geo::kTok, er.p1 - pc);
         for (int i = 0; i < nt; ++i) {
             const size_t p = static_cast<size_t>(pc + i);
             stage_act_row<QT>(qh + p * I, dh + p * nb, nb, a0 + i * nb, a1 + i * nb, ad + i * nb,
                               as + i * nb, threadIdx.x, kThreads);
         }
-        const int t0 = warp * kDownTpw, ntw = min(kDownTpw, nt - t0);
-        float acc[kDownTpw];
+        const int t0 = pg * kTpw, ntw = min(kTpw, nt - t0);
+        float acc[kTpw];
 #pragma unroll
-        for (int t = 0; t < kDownTpw; ++t) acc[t] = 0.0f;
+        for (int t = 0; t < kTpw; ++t) acc[t] = 0.0f;
         Chunk wc;
         wc.load(row_ptr, rb, 0);
         for (int c = 0; c < nchunks; ++c) {
@@ -259,18 +286,19 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
             wc.store(wsm);
             __syncthreads();
             if (c + 1 < nchunks) wc.load(row_ptr, rb, c + 1);
+            const int b0 = c * Chunk::kChunkBlocks;
             if (ntw > 0)
-                row_dots_chunk<QT, kDownTpw>(wrow, c * kCB, min(kCB, nb - c * kCB), nb, a0, a1, ad, as, t0, ntw,
-                                             sg, gs / 32, acc);
+                row_dots_chunk<QT, kTpw>(wrow, b0, min(Chunk::kChunkBlocks, nb - b0), nb, a0, a1, ad, as, t0, ntw,
+                                         sg, gs / 32, acc);
         }
         if (ntw > 0) {
 #pragma unroll
-            for (int t = 0; t < kDownTpw; ++t) {
+            for (int t = 0; t < kTpw; ++t) {
                 if (t < ntw) {
                     const int p = pc + t0 + t;
                     const int tok = un.uniq ? un.pair_tok[p] : p;
                     const int slot = un.uniq ? un.pair_slot[p] : 0;
-                    y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + lane] = gs ? acc[t] : __fmul_rn(acc[t], srow);
+                    y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + orow] = gs ? acc[t] : __fmul_rn(acc[t], srow);
                 }
             }
         }
@@ -278,30 +306,32 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
     }
 }
 
-template <int QT>
+template <int QT, bool W>
 cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
                        const UnionView& un, int8_t* qh, float* dh, cudaStream_t st) {
+    using Geo = UgGeom<W>;
     const int nb = ex.hidden / 32;
-    const size_t smem = WeightChunk<QT, 2 * kUgRows>::kBytes + static_cast<size_t>(kUgTok) * nb * 40 +
-                        2 * kUgTok * kUgRows * sizeof(float);
-    auto kern = k_up_gate<QT>;
+    const size_t smem = ChunkOf<QT, 2 * Geo::kRows, W>::kBytes + static_cast<size_t>(Geo::kTok) * nb * 40 +
+                        2 * Geo::kTok * Geo::kRows * sizeof(float);
+    auto kern = k_up_gate<QT, W>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(ex.inter / kUgRows, un.max_unique);
+    const dim3 grid(ex.inter / Geo::kRows, un.max_unique);
     kern<<<grid, kThreads, smem, st>>>(ex.w_gate, ex.w_up, ex.s_gate, ex.s_up, ex.hidden, ex.inter,
                                        ex.group_size, qx, dx, T, un, qh, dh);
     return counted(cudaGetLastError());
 }
 
-template <int QT>
+template <int QT, bool W>
 cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, int T, int K,
                     const UnionView& un, float* y, cudaStream_t st) {
+    using Geo = DownGeom<W>;
     const int nb = ex.inter / 32;
-    const size_t smem = WeightChunk<QT, kDownRows>::kBytes + static_cast<size_t>(kDownTok) * nb * 40;
-    auto kern = k_down<QT>;
+    const size_t smem = ChunkOf<QT, Geo::kRows, W>::kBytes + static_cast<size_t>(Geo::kTok) * nb * 40;
+    auto kern = k_down<QT, W>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(ex.hidden / kDownRows, un.max_unique);
+    const dim3 grid(ex.hidden / Geo::kRows, un.max_unique);
     kern<<<grid, kThreads, smem, st>>>(ex.w_down, ex.s_down, ex.hidden, ex.inter, ex.group_size, qh, dh, T, K,
                                        un, y);
     return counted(cudaGetLastError());
@@ -310,23 +340,32 @@ cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, in
 }  // namespace
 
 cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
-                                  const UnionView& un, int8_t* qh, float* dh, cudaStream_t st) {
+                                  const UnionView& un, int tok_per_expert, int8_t* qh, float* dh,
+                                  cudaStream_t st) {
     if (un.max_unique <= 0) return cudaSuccess;
+    const bool wide = tok_per_expert <= kTpw && ex.inter % UgGeom<true>::kRows == 0;
     switch (ex.qtype) {
-        case MOE_Q_INT4: return up_gate_qt<4>(ex, qx, dx, T, un, qh, dh, st);
-        case MOE_Q_INT8: return up_gate_qt<8>(ex, qx, dx, T, un, qh, dh, st);
-        case MOE_Q_INT2: return up_gate_qt<2>(ex, qx, dx, T, un, qh, dh, st);
+        case MOE_Q_INT4: return wide ? up_gate_qt<4, true>(ex, qx, dx, T, un, qh, dh, st)
+                                     : up_gate_qt<4, false>(ex, qx, dx, T, un, qh, dh, st);
+        case MOE_Q_INT8: return wide ? up_gate_qt<8, true>(ex, qx, dx, T, un, qh, dh, st)
+                                     : up_gate_qt<8, false>(ex, qx, dx, T, un, qh, dh, st);
+        case MOE_Q_INT2: return wide ? up_gate_qt<2, true>(ex, qx, dx, T, un, qh, dh, st)
+                                     : up_gate_qt<2, false>(ex, qx, dx, T, un, qh, dh, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
-                               int top_k, const UnionView& un, float* y, cudaStream_t st) {
+                               int top_k, const UnionView& un, int tok_per_expert, float* y, cudaStream_t st) {
     if (un.max_unique <= 0) return cudaSuccess;
+    const bool wide = tok_per_expert <= kTpw && ex.hidden % DownGeom<true>::kRows == 0;
     switch (ex.qtype) {
-        case MOE_Q_INT4: return down_qt<4>(ex, qh, dh, T, top_k, un, y, st);
-        case MOE_Q_INT8: return down_qt<8>(ex, qh, dh, T, top_k, un, y, st);
-        case MOE_Q_INT2: return down_qt<2>(ex, qh, dh, T, top_k, un, y, st);
+        case MOE_Q_INT4: return wide ? down_qt<4, true>(ex, qh, dh, T, top_k, un, y, st)
+                                     : down_qt<4, false>(ex, qh, dh, T, top_k, un, y, st);
+        case MOE_Q_INT8: return wide ? down_qt<8, true>(ex, qh, dh, T, top_k, un, y, st)
+                                     : down_qt<8, false>(ex, qh, dh, T, top_k, un, y, st);
+        case MOE_Q_INT2: return wide ? down_qt<2, true>(ex, qh, dh, T, top_k, un, y, st)
+                                     : down_qt<2, false>(ex, qh, dh, T, top_k, un, y, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -46,12 +46,22 @@ struct UnionView {
     int max_unique;  // grid bound (device value n_unique <= max_unique)
 };
 
+// Tokens each expert of a union sees on average (rounded up): it picks the
+// general path kernels' CTA geometry.  A dense view (uniq null) is one expert
+// seeing all T tokens.
+inline int tokens_per_expert(const UnionView& un, int T, int top_k) {
+    if (!un.uniq) return T;
+    const long long pairs = static_cast<long long>(T) * top_k;
+    return static_cast<int>((pairs + un.max_unique - 1) / un.max_unique);
+}
 // up/gate + SwiGLU + Q8_0(h) for every pair; qh [P][I], dh [P][I/32] by pair index.
 cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
-                                  const UnionView& un, int8_t* qh, float* dh, cudaStream_t st);
+                                  const UnionView& un, int tok_per_expert, int8_t* qh, float* dh,
+                                  cudaStream_t st);
 // down rows for every pair, written to y_pairs[tok][slot][:].
 cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
-                               int top_k, const UnionView& un, float* y_pairs, cudaStream_t st);
+                               int top_k, const UnionView& un, int tok_per_expert, float* y_pairs,
+                               cudaStream_t st);
 
 cudaError_t launch_usage_accumulate(const int32_t* idx, long n, int E, uint32_t* usage, cudaStream_t st);
 cudaError_t launch_usage_rank(const uint32_t* usage, int E, int32_t* order, cudaStream_t st);
