@@ -159,7 +159,7 @@ __device__ __forceinline__ void row_dots_chunk(const uint8_t* row, int b0, int n
 }
 
 template <int QT, bool W>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, QT == 4 ? 2 : 1)  // int4: two CTAs an SM (measured 3% faster)
 k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
           const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I, int gs,
           const int8_t* __restrict__ qx, const float* __restrict__ dx, int T, UnionView un,
@@ -239,7 +239,7 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
 }
 
 template <int QT, bool W>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, QT == 4 ? 2 : 1)  // int4: two CTAs an SM (measured 3% faster)
 k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I, int gs,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
        float* __restrict__ y_pairs) {
