@@ -109,6 +109,13 @@ def parse():
                          "clocks are sampled")
     ap.add_argument("--prefill-only", action="store_true",
                     help="run only the prefill measurement and print its entry (for profiler captures)")
+    ap.add_argument("--layer-calls", default=None, metavar="CONFIG",
+                    help="run only a few layer calls of a named workload (synth.CONFIGS; for profiler "
+                         "captures) and print the path taken and the time per call")
+    ap.add_argument("--layer-tokens", type=int, default=0, help="--layer-calls: tokens per call (0: the config's)")
+    ap.add_argument("--layer-experts", type=int, default=0,
+                    help="--layer-calls: routed experts (0: the config's; otherwise in 8 groups, top-4 groups)")
+    ap.add_argument("--layer-reps", type=int, default=8, help="--layer-calls: calls made")
     return ap.parse_args()
 
 
@@ -135,6 +142,34 @@ def oracle_sample(sh, seconds: float, first_token: int = 0, max_tokens: int | No
     return dict(value=n * sh.T / total, unit="tokens/s", cores=threads, kind="oracle",
                 sample=f"{n} decode tokens (T=1 layer calls, each routed afresh), "
                        f"{total:.1f} s of oracle time; weight generation excluded"), n, total
+
+
+def layer_calls(args, moe, device_layer, to_dev_bf16):
+    """A few back-to-back layer calls of one workload, one resident layer (profiler captures)."""
+    import torch
+    sh = synth.CONFIGS[args.layer_calls].with_(n_layers=1)
+    if args.layer_tokens:
+        sh = sh.with_(T=args.layer_tokens)
+    if args.layer_experts:
+        sh = sh.with_(E=args.layer_experts, n_group=8, topk_group=4)
+    dev = device_layer(sh)
+    x = to_dev_bf16(synth.hidden_states(sh, tokens=range(sh.T)))
+    out = torch.empty(sh.T, sh.H, dtype=torch.bfloat16, device="cuda")
+    ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
+    path = moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"])
+    moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)  # warm-up
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.layer_reps):
+        moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    if moe.moe_workspace_status(ws) != 0:
+        raise RuntimeError("device status error during the layer calls")
+    return {"workload": f"{sh.name}: T={sh.T}, {sh.E} routed experts, {sh.qtype}-bit, one resident layer",
+            "path": {moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core", moe.PATH_GENERAL: "general"}[path],
+            "calls": args.layer_reps, "ms_per_call": e0.elapsed_time(e1) / max(args.layer_reps, 1),
+            "device_GB": torch.cuda.max_memory_allocated() / 1e9}
 
 
 def run_reference(args):
@@ -503,6 +538,10 @@ def run_cuda(args):
     if args.prefill_only:
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
         print(json.dumps(prefill_measurement(args, moe, moe.lib(), device_layer, to_dev_bf16)), flush=True)
+        return
+    if args.layer_calls:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(layer_calls(args, moe, device_layer, to_dev_bf16)), flush=True)
         return
 
     world, rank, local = rank_env()
