@@ -145,7 +145,8 @@ def oracle_sample(sh, seconds: float, first_token: int = 0, max_tokens: int | No
 
 
 def layer_calls(args, moe, device_layer, to_dev_bf16):
-    """A few back-to-back layer calls of one workload, one resident layer (profiler captures)."""
+    """A few back-to-back layer calls of one workload, one resident layer (profiler captures; the
+    time per call includes the first call's one-time setup)."""
     import torch
     sh = synth.CONFIGS[args.layer_calls].with_(n_layers=1)
     if args.layer_tokens:
@@ -157,7 +158,6 @@ def layer_calls(args, moe, device_layer, to_dev_bf16):
     out = torch.empty(sh.T, sh.H, dtype=torch.bfloat16, device="cuda")
     ws = moe.workspace(moe.moe_layer_workspace_bytes(sh.T, dev["cfg"], dev["routed"], dev["shared"]))
     path = moe.moe_layer_path(sh.T, dev["cfg"], dev["routed"], dev["shared"])
-    moe.moe_layer_forward(x, dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], out, ws)  # warm-up
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.layer_reps):
