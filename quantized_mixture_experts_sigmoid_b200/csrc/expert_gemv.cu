@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, QT == 4 ? 2 : 1)  // int4: two CTAs 
 k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
           const float* __restrict__ s_gate, const float* __restrict__ s_up, int H, int I, int gs,
           const int8_t* __restrict__ qx, const float* __restrict__ dx, int T, UnionView un,
-          int8_t* __restrict__ qh, float* __restrict__ dh) {
+          int8_t* __restrict__ qh, float* __restrict__ dh, SharedUpGate sx) {
     using Geo = UgGeom<W>;
     using Chunk = ChunkOf<QT, 2 * Geo::kRows, W>;  // the CTA's gate rows, then its up rows
     extern __shared__ __align__(16) uint8_t smem[];
@@ -176,8 +176,17 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     float* gbuf = reinterpret_cast<float*>(as + Geo::kTok * nb);
     float* ubuf = gbuf + Geo::kTok * Geo::kRows;
 
+    // grid row 0 is the shared expert when it rides along (all T tokens), the
+    // others the union's experts
+    const bool shared = sx.w_gate && blockIdx.y == 0;
     ExpertRange er;
-    if (!expert_range(un, blockIdx.y, T, er)) return;
+    if (shared) {
+        er = ExpertRange{0, 0, T};
+        w_gate = sx.w_gate; w_up = sx.w_up; s_gate = sx.s_gate; s_up = sx.s_up; qh = sx.qh; dh = sx.dh;
+    } else if (!expert_range(un, blockIdx.y - (sx.w_gate ? 1 : 0), T, er)) {
+        return;
+    }
+    const bool dense = shared || !un.uniq;  // rows are tokens, not union pairs
     const int r0 = blockIdx.x * Geo::kRows;
     const size_t rb = static_cast<size_t>(H) * QT / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,7 +206,7 @@ k_up_gate(const uint8_t* __restrict__ w_gate, const uint8_t* __restrict__ w_up,
     for (int pc = er.p0; pc < er.p1; pc += Geo::kTok) {
         const int nt = min(Geo::kTok, er.p1 - pc);
         for (int i = 0; i < nt; ++i) {
-            const int tok = un.uniq ? un.pair_tok[pc + i] : pc + i;
+            const int tok = dense ? pc + i : un.pair_tok[pc + i];
             stage_act_row<QT>(qx + static_cast<size_t>(tok) * H, dx + static_cast<size_t>(tok) * nb,
                               nb, a0 + i * nb, a1 + i * nb, ad + i * nb, as + i * nb, threadIdx.x,
                               kThreads);
@@ -242,7 +251,7 @@ template <int QT, bool W>
 __global__ void __launch_bounds__(kThreads, QT == 4 ? 2 : 1)  // int4: two CTAs an SM (measured 3% faster)
 k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int H, int I, int gs,
        const int8_t* __restrict__ qh, const float* __restrict__ dh, int T, int K, UnionView un,
-       float* __restrict__ y_pairs) {
+       float* __restrict__ y_pairs, SharedDown sx) {
     using Geo = DownGeom<W>;
     using Chunk = ChunkOf<QT, Geo::kRows, W>;
     extern __shared__ __align__(16) uint8_t smem[];
@@ -253,8 +262,16 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
     float* ad = reinterpret_cast<float*>(a1 + Geo::kTok * nb);
     int32_t* as = reinterpret_cast<int32_t*>(ad + Geo::kTok * nb);
 
+    // grid row 0 is the shared expert when it rides along (all T tokens, one slot)
+    const bool shared = sx.w_down && blockIdx.y == 0;
     ExpertRange er;
-    if (!expert_range(un, blockIdx.y, T, er)) return;
+    if (shared) {
+        er = ExpertRange{0, 0, T};
+        w_down = sx.w_down; s_down = sx.s_down; qh = sx.qh; dh = sx.dh; y_pairs = sx.y; K = 1;
+    } else if (!expert_range(un, blockIdx.y - (sx.w_down ? 1 : 0), T, er)) {
+        return;
+    }
+    const bool dense = shared || !un.uniq;  // rows are tokens, not union pairs
     const int c0 = blockIdx.x * Geo::kRows;
     const size_t rb = static_cast<size_t>(I) * QT / 8;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,8 +313,8 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
             for (int t = 0; t < kTpw; ++t) {
                 if (t < ntw) {
                     const int p = pc + t0 + t;
-                    const int tok = un.uniq ? un.pair_tok[p] : p;
-                    const int slot = un.uniq ? un.pair_slot[p] : 0;
+                    const int tok = dense ? p : un.pair_tok[p];
+                    const int slot = dense ? 0 : un.pair_slot[p];
                     y_pairs[(static_cast<size_t>(tok) * K + slot) * H + c0 + orow] = gs ? acc[t] : __fmul_rn(acc[t], srow);
                 }
             }
@@ -308,7 +325,7 @@ k_down(const uint8_t* __restrict__ w_down, const float* __restrict__ s_down, int
 
 template <int QT, bool W>
 cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
-                       const UnionView& un, int8_t* qh, float* dh, cudaStream_t st) {
+                       const UnionView& un, int8_t* qh, float* dh, const SharedUpGate& sx, cudaStream_t st) {
     using Geo = UgGeom<W>;
     const int nb = ex.hidden / 32;
     const size_t smem = ChunkOf<QT, 2 * Geo::kRows, W>::kBytes + static_cast<size_t>(Geo::kTok) * nb * 40 +
@@ -316,24 +333,24 @@ cudaError_t up_gate_qt(const moe_experts& ex, const int8_t* qx, const float* dx,
     auto kern = k_up_gate<QT, W>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(ex.inter / Geo::kRows, un.max_unique);
+    const dim3 grid(ex.inter / Geo::kRows, un.max_unique + (sx.w_gate ? 1 : 0));
     kern<<<grid, kThreads, smem, st>>>(ex.w_gate, ex.w_up, ex.s_gate, ex.s_up, ex.hidden, ex.inter,
-                                       ex.group_size, qx, dx, T, un, qh, dh);
+                                       ex.group_size, qx, dx, T, un, qh, dh, sx);
     return counted(cudaGetLastError());
 }
 
 template <int QT, bool W>
 cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, int T, int K,
-                    const UnionView& un, float* y, cudaStream_t st) {
+                    const UnionView& un, float* y, const SharedDown& sx, cudaStream_t st) {
     using Geo = DownGeom<W>;
     const int nb = ex.inter / 32;
     const size_t smem = ChunkOf<QT, Geo::kRows, W>::kBytes + static_cast<size_t>(Geo::kTok) * nb * 40;
     auto kern = k_down<QT, W>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid(ex.hidden / Geo::kRows, un.max_unique);
+    const dim3 grid(ex.hidden / Geo::kRows, un.max_unique + (sx.w_down ? 1 : 0));
     kern<<<grid, kThreads, smem, st>>>(ex.w_down, ex.s_down, ex.hidden, ex.inter, ex.group_size, qh, dh, T, K,
-                                       un, y);
+                                       un, y, sx);
     return counted(cudaGetLastError());
 }
 
@@ -341,31 +358,32 @@ cudaError_t down_qt(const moe_experts& ex, const int8_t* qh, const float* dh, in
 
 cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
                                   const UnionView& un, int tok_per_expert, int8_t* qh, float* dh,
-                                  cudaStream_t st) {
-    if (un.max_unique <= 0) return cudaSuccess;
+                                  const SharedUpGate& sx, cudaStream_t st) {
+    if (un.max_unique <= 0 && !sx.w_gate) return cudaSuccess;
     const bool wide = tok_per_expert <= kTpw && ex.inter % UgGeom<true>::kRows == 0;
     switch (ex.qtype) {
-        case MOE_Q_INT4: return wide ? up_gate_qt<4, true>(ex, qx, dx, T, un, qh, dh, st)
-                                     : up_gate_qt<4, false>(ex, qx, dx, T, un, qh, dh, st);
-        case MOE_Q_INT8: return wide ? up_gate_qt<8, true>(ex, qx, dx, T, un, qh, dh, st)
-                                     : up_gate_qt<8, false>(ex, qx, dx, T, un, qh, dh, st);
-        case MOE_Q_INT2: return wide ? up_gate_qt<2, true>(ex, qx, dx, T, un, qh, dh, st)
-                                     : up_gate_qt<2, false>(ex, qx, dx, T, un, qh, dh, st);
+        case MOE_Q_INT4: return wide ? up_gate_qt<4, true>(ex, qx, dx, T, un, qh, dh, sx, st)
+                                     : up_gate_qt<4, false>(ex, qx, dx, T, un, qh, dh, sx, st);
+        case MOE_Q_INT8: return wide ? up_gate_qt<8, true>(ex, qx, dx, T, un, qh, dh, sx, st)
+                                     : up_gate_qt<8, false>(ex, qx, dx, T, un, qh, dh, sx, st);
+        case MOE_Q_INT2: return wide ? up_gate_qt<2, true>(ex, qx, dx, T, un, qh, dh, sx, st)
+                                     : up_gate_qt<2, false>(ex, qx, dx, T, un, qh, dh, sx, st);
         default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
-                               int top_k, const UnionView& un, int tok_per_expert, float* y, cudaStream_t st) {
-    if (un.max_unique <= 0) return cudaSuccess;
+                               int top_k, const UnionView& un, int tok_per_expert, float* y,
+                               const SharedDown& sx, cudaStream_t st) {
+    if (un.max_unique <= 0 && !sx.w_down) return cudaSuccess;
     const bool wide = tok_per_expert <= kTpw && ex.hidden % DownGeom<true>::kRows == 0;
     switch (ex.qtype) {
-        case MOE_Q_INT4: return wide ? down_qt<4, true>(ex, qh, dh, T, top_k, un, y, st)
-                                     : down_qt<4, false>(ex, qh, dh, T, top_k, un, y, st);
-        case MOE_Q_INT8: return wide ? down_qt<8, true>(ex, qh, dh, T, top_k, un, y, st)
-                                     : down_qt<8, false>(ex, qh, dh, T, top_k, un, y, st);
-        case MOE_Q_INT2: return wide ? down_qt<2, true>(ex, qh, dh, T, top_k, un, y, st)
-                                     : down_qt<2, false>(ex, qh, dh, T, top_k, un, y, st);
+        case MOE_Q_INT4: return wide ? down_qt<4, true>(ex, qh, dh, T, top_k, un, y, sx, st)
+                                     : down_qt<4, false>(ex, qh, dh, T, top_k, un, y, sx, st);
+        case MOE_Q_INT8: return wide ? down_qt<8, true>(ex, qh, dh, T, top_k, un, y, sx, st)
+                                     : down_qt<8, false>(ex, qh, dh, T, top_k, un, y, sx, st);
+        case MOE_Q_INT2: return wide ? down_qt<2, true>(ex, qh, dh, T, top_k, un, y, sx, st)
+                                     : down_qt<2, false>(ex, qh, dh, T, top_k, un, y, sx, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -54,14 +54,32 @@ inline int tokens_per_expert(const UnionView& un, int T, int top_k) {
     const long long pairs = static_cast<long long>(T) * top_k;
     return static_cast<int>((pairs + un.max_unique - 1) / un.max_unique);
 }
+// A shared expert of the routed experts' shape computed in the same launch
+// (grid row 0, all T tokens): its weights and outputs; w_gate / w_down null
+// when there is none.
+struct SharedUpGate {
+    const uint8_t* w_gate;
+    const uint8_t* w_up;
+    const float* s_gate;
+    const float* s_up;
+    int8_t* qh;  // [T][I]
+    float* dh;   // [T][I/32]
+};
+struct SharedDown {
+    const uint8_t* w_down;
+    const float* s_down;
+    const int8_t* qh;  // [T][I]
+    const float* dh;   // [T][I/32]
+    float* y;          // [T][H]
+};
 // up/gate + SwiGLU + Q8_0(h) for every pair; qh [P][I], dh [P][I/32] by pair index.
 cudaError_t launch_expert_up_gate(const moe_experts& ex, const int8_t* qx, const float* dx, int T,
                                   const UnionView& un, int tok_per_expert, int8_t* qh, float* dh,
-                                  cudaStream_t st);
+                                  const SharedUpGate& sx, cudaStream_t st);
 // down rows for every pair, written to y_pairs[tok][slot][:].
 cudaError_t launch_expert_down(const moe_experts& ex, const int8_t* qh, const float* dh, int T,
                                int top_k, const UnionView& un, int tok_per_expert, float* y_pairs,
-                               cudaStream_t st);
+                               const SharedDown& sx, cudaStream_t st);
 
 cudaError_t launch_usage_accumulate(const int32_t* idx, long n, int E, uint32_t* usage, cudaStream_t st);
 cudaError_t launch_usage_rank(const uint32_t* usage, int E, int32_t* order, cudaStream_t st);
