@@ -1,0 +1,112 @@
+"""Expert parallelism across ranks (the routed experts split by expert, one
+all-to-all each way): two gloo ranks on the CPU, each with its own tokens and
+half of the experts, the compute steps given by the oracle; every rank's
+output rows equal the single-process oracle layer's bit for bit, with and
+without adaptive top-p (empty slots are not sent).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import synth
+
+SHAPE = synth.LayerShape("ep_small", T=7, H=256, I=128, E=16, n_group=4, topk_group=2, top_k=4)
+
+
+def _port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _oracle_compute(sh, top_p, rank, n_ranks):
+    from oracle import oracle as O
+    from oracle.synth_inputs import oracle_experts
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import EPCompute
+
+    W, b = synth.router_weight(sh), synth.router_bias(sh)
+    per = sh.E // n_ranks
+    routed = oracle_experts(sh, range(rank * per, (rank + 1) * per))  # this rank's experts only
+    shared = oracle_experts(sh, [0], shared=True)
+
+    def bits(t):
+        return t.view(torch.int16).numpy().view(np.uint16)
+
+    def route(x):
+        idx, w, _, _ = O.route(bits(x), W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf, top_p)
+        return torch.from_numpy(idx.astype(np.int32)), torch.from_numpy(w.astype(np.float32))
+
+    def experts(rows, local_idx):
+        gidx = (local_idx.numpy().astype(np.int32) + rank * per).reshape(-1, 1)
+        return torch.from_numpy(O.expert_ffn_per_token(routed, bits(rows), gidx)[:, 0, :].copy())
+
+    def shared_fn(x):
+        zero = np.zeros((x.shape[0], 1), dtype=np.int32)
+        return torch.from_numpy(O.expert_ffn_per_token(shared, bits(x), zero)[:, 0, :].copy())
+
+    def combine(y_pairs, w, shared_y):
+        of, _ = O.combine(y_pairs.numpy(), w.numpy(), None if shared_y is None else shared_y.numpy())
+        return torch.from_numpy(of)
+
+    return EPCompute(route, experts, shared_fn, combine)
+
+
+def _rank_main(rank, n_ranks, port, top_p, splits, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=n_ranks, timeout=datetime.timedelta(seconds=60))
+    try:
+        from quantized_mixture_experts_sigmoid_b200.expert_parallel import ep_forward
+        x = synth.hidden_states(SHAPE)
+        t0, t1 = splits[rank], splits[rank + 1]
+        xr = torch.from_numpy(x[t0:t1].view(np.int16).copy()).view(torch.bfloat16)
+        out = ep_forward(xr, SHAPE.E, _oracle_compute(SHAPE, top_p, rank, n_ranks))
+        q.put((rank, out.numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _reference(top_p):
+    from oracle import oracle as O
+    from oracle.synth_inputs import oracle_experts
+    x = synth.hidden_states(SHAPE)
+    W, b = synth.router_weight(SHAPE), synth.router_bias(SHAPE)
+    routed = oracle_experts(SHAPE, range(SHAPE.E))
+    shared = oracle_experts(SHAPE, [0], shared=True)
+    of, _, idx, _ = O.layer_forward(x, W, b, SHAPE.n_group, SHAPE.topk_group, SHAPE.top_k, SHAPE.rsf,
+                                    routed, shared, top_p)
+    return of, idx
+
+
+@pytest.mark.parametrize("top_p", [0.0, 0.6])
+def test_two_ranks_equal_one_process(top_p):
+    splits = [0, 4, SHAPE.T]  # ragged: 4 and 3 tokens
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, top_p, splits, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        got = dict(q.get(timeout=60) for _ in procs)
+        for p in procs:
+            p.join(timeout=60)
+            assert p.exitcode == 0
+    finally:
+        for p in procs:  # a rank that failed leaves the other waiting in a collective
+            if p.is_alive():
+                p.kill()
+    ref, idx = _reference(top_p)
+    if top_p:
+        assert (idx < 0).any()  # some slots are empty and go nowhere
+    per = SHAPE.E // 2
+    assert ((idx >= per) & (np.arange(SHAPE.T)[:, None] < 4)).any()  # rank 0 sends to rank 1
+    assert ((idx >= 0) & (idx < per) & (np.arange(SHAPE.T)[:, None] >= 4)).any()  # and back
+    for r in range(2):
+        assert np.array_equal(got[r].view(np.uint32), ref[splits[r]:splits[r + 1]].view(np.uint32))
