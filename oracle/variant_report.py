@@ -10,7 +10,7 @@ moe_oracle.c's compile-time switches build the three other combinations:
   "muladd"        fold acc = acc + isum * d (two roundings)
   "silu32_muladd" both
 
-For seeded inputs of the spec workloads this script routes every token
+For seeded inputs of the measured workloads this script routes every token
 with the default oracle (routing uses neither rounding), evaluates every
 (token, expert) pair under all four variants and reports, against the
 default: h elements that differ, Q8_0(h) codes that flip, and the layer
