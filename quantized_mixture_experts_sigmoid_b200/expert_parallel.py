@@ -19,6 +19,12 @@ Empty slots (index -1: adaptive top-p) are not sent and add nothing.  Each
 pair's output is the same expert function of the same token row on any rank,
 and step 5 sums in slot order, so the result equals the single-GPU layer's.
 
+Which rank holds which expert is a placement: contiguous slices by default,
+or `placement_by_usage`, which deals the experts out in the usage record's
+most-used-first order ([HN] "Learning cache와 하드웨어별 기대치": the hottest
+experts are the ones worth placing) so every rank gets an even share of the
+hot ones and of the routed pairs.
+
 The exchange is plain collectives (NCCL between GPUs); the compute steps are
 this library's C-ABI calls (`ep_cuda_compute`) or, in tests, any functions of
 the same signatures.
@@ -47,13 +53,48 @@ class EPCompute:
     combine: Callable
 
 
+def placement_by_usage(order: torch.Tensor, n_ranks: int) -> tuple[torch.Tensor, torch.Tensor]:
+    """Expert placement from a most-used-first order (moe_usage_rank's output).
+
+    Deals the experts to the ranks in that order, turning at the ends (0, 1, .., N-1, N-1, .., 0,
+    0, 1, ..), so each rank holds E / N experts and a near-even share of the usage.  Returns
+    (owner [E]: the rank holding each expert, local [E]: its index among that rank's experts,
+    which are numbered in dealing order).
+    """
+    order = order.to(torch.int64).cpu()
+    E = order.numel()
+    if E % n_ranks:
+        raise ValueError(f"{E} experts do not split evenly over {n_ranks} ranks")
+    owner = torch.empty(E, dtype=torch.int64)
+    local = torch.empty(E, dtype=torch.int64)
+    filled = [0] * n_ranks
+    for i, e in enumerate(order.tolist()):
+        lap, pos = divmod(i, n_ranks)
+        r = pos if lap % 2 == 0 else n_ranks - 1 - pos
+        owner[e] = r
+        local[e] = filled[r]
+        filled[r] += 1
+    return owner, local
+
+
+def experts_of_rank(owner: torch.Tensor, local: torch.Tensor, rank: int) -> torch.Tensor:
+    """The global indices of the experts `rank` holds, in local-index order."""
+    mine = torch.nonzero(owner.cpu() == rank).flatten()
+    return mine[torch.argsort(local.cpu()[mine])]
+
+
 def _a2a(out: torch.Tensor, inp: torch.Tensor, out_splits, in_splits, group) -> torch.Tensor:
     dist.all_to_all_single(out, inp, output_split_sizes=out_splits, input_split_sizes=in_splits, group=group)
     return out
 
 
-def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None) -> torch.Tensor:
-    """One expert-parallel layer call on this rank's tokens x [T, H] (bf16)."""
+def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None,
+               placement: tuple[torch.Tensor, torch.Tensor] | None = None) -> torch.Tensor:
+    """One expert-parallel layer call on this rank's tokens x [T, H] (bf16).
+
+    placement: (owner [E], local [E]) as from placement_by_usage, the same on every rank; None for
+    contiguous slices (rank r holds experts r E/N .. (r+1) E/N - 1).
+    """
     n = dist.get_world_size(group)
     if n_expert % n:
         raise ValueError(f"{n_expert} experts do not split evenly over {n} ranks")
@@ -63,7 +104,15 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None) -
     K = idx.shape[1]
     flat = idx.reshape(-1).to(torch.int64)
     valid = flat >= 0
-    dest = torch.where(valid, flat // per, torch.full_like(flat, n))  # empty slots sort last, go nowhere
+    if placement is None:
+        owner_of = torch.where(valid, flat // per, torch.full_like(flat, n))
+        local_of = flat - owner_of * per
+    else:
+        owner, loc = (t.to(device=x.device, dtype=torch.int64) for t in placement)
+        safe = torch.where(valid, flat, torch.zeros_like(flat))
+        owner_of = torch.where(valid, owner[safe], torch.full_like(flat, n))
+        local_of = loc[safe]
+    dest = owner_of  # empty slots (rank n) sort last and go nowhere
     order = torch.argsort(dest, stable=True)  # pairs by destination rank, (token, slot) ascending within
     n_send = int(valid.sum())
     order = order[:n_send]
@@ -75,7 +124,7 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None) -
 
     # the pairs' token rows as raw bf16 bits, two to a 32-bit word (H is even)
     rows = x.contiguous().view(torch.int32).index_select(0, order // K)
-    local = (flat[order] - dest[order] * per).to(torch.int32)  # expert index on the destination rank
+    local = local_of[order].to(torch.int32)  # expert index on the destination rank
     recv_rows = _a2a(torch.empty(n_recv, H // 2, dtype=torch.int32, device=x.device), rows, rc, sc, group)
     recv_local = _a2a(torch.empty(n_recv, dtype=torch.int32, device=x.device), local, rc, sc, group)
 
@@ -90,17 +139,26 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None) -
 
 
 def ep_cuda_compute(w_router: torch.Tensor, bias: torch.Tensor, cfg, routed, shared=None,
-                    rank: int = 0, n_ranks: int = 1, out_dtype=torch.bfloat16) -> EPCompute:
+                    rank: int = 0, n_ranks: int = 1, out_dtype=torch.bfloat16,
+                    placement: tuple[torch.Tensor, torch.Tensor] | None = None) -> EPCompute:
     """EPCompute on this library's kernels for rank `rank` of `n_ranks`.
 
-    routed: the full stacked ExpertSet (all E experts; this rank uses its slice), or an ExpertSet
-    already holding only the rank's E / n_ranks experts.  shared: ExpertSet of one expert or None.
+    routed: the full stacked ExpertSet (all E experts; this rank uses its share), or an ExpertSet
+    already holding only the rank's E / n_ranks experts in local-index order.  shared: ExpertSet
+    of one expert or None.  placement: as for ep_forward (the rank's experts are gathered into a
+    stack of their own when it is given with the full set).
     """
     from . import moe
 
     E = cfg.n_expert
     per = E // n_ranks
-    if routed.n_expert == E:
+    if placement is not None and routed.n_expert == E:
+        mine = experts_of_rank(*placement, rank).to(routed.w_gate.device)
+        pick = lambda t: t.index_select(0, mine).contiguous()  # noqa: E731
+        local = moe.ExpertSet(routed.qtype, per, routed.hidden, routed.inter, pick(routed.w_gate),
+                              pick(routed.w_up), pick(routed.w_down), pick(routed.s_gate), pick(routed.s_up),
+                              pick(routed.s_down), routed.group_size)
+    elif routed.n_expert == E:
         e0, e1 = rank * per, (rank + 1) * per
         local = moe.ExpertSet(routed.qtype, per, routed.hidden, routed.inter, routed.w_gate[e0:e1],
                               routed.w_up[e0:e1], routed.w_down[e0:e1], routed.s_gate[e0:e1],

@@ -24,14 +24,18 @@ def _port():
         return s.getsockname()[1]
 
 
-def _oracle_compute(sh, top_p, rank, n_ranks):
+def _oracle_compute(sh, top_p, rank, n_ranks, placement=None):
     from oracle import oracle as O
     from oracle.synth_inputs import oracle_experts
-    from quantized_mixture_experts_sigmoid_b200.expert_parallel import EPCompute
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import EPCompute, experts_of_rank
 
     W, b = synth.router_weight(sh), synth.router_bias(sh)
     per = sh.E // n_ranks
-    routed = oracle_experts(sh, range(rank * per, (rank + 1) * per))  # this rank's experts only
+    if placement is None:
+        mine = np.arange(rank * per, (rank + 1) * per)
+    else:
+        mine = experts_of_rank(*placement, rank).numpy()
+    routed = oracle_experts(sh, mine)  # this rank's experts only
     shared = oracle_experts(sh, [0], shared=True)
 
     def bits(t):
@@ -42,7 +46,7 @@ def _oracle_compute(sh, top_p, rank, n_ranks):
         return torch.from_numpy(idx.astype(np.int32)), torch.from_numpy(w.astype(np.float32))
 
     def experts(rows, local_idx):
-        gidx = (local_idx.numpy().astype(np.int32) + rank * per).reshape(-1, 1)
+        gidx = mine[local_idx.numpy()].astype(np.int32).reshape(-1, 1)
         return torch.from_numpy(O.expert_ffn_per_token(routed, bits(rows), gidx)[:, 0, :].copy())
 
     def shared_fn(x):
@@ -56,7 +60,7 @@ def _oracle_compute(sh, top_p, rank, n_ranks):
     return EPCompute(route, experts, shared_fn, combine)
 
 
-def _rank_main(rank, n_ranks, port, top_p, splits, q):
+def _rank_main(rank, n_ranks, port, top_p, splits, q, usage_placement=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     import datetime
@@ -66,10 +70,22 @@ def _rank_main(rank, n_ranks, port, top_p, splits, q):
         x = synth.hidden_states(SHAPE)
         t0, t1 = splits[rank], splits[rank + 1]
         xr = torch.from_numpy(x[t0:t1].view(np.int16).copy()).view(torch.bfloat16)
-        out = ep_forward(xr, SHAPE.E, _oracle_compute(SHAPE, top_p, rank, n_ranks))
+        placement = _usage_placement(n_ranks) if usage_placement else None
+        out = ep_forward(xr, SHAPE.E, _oracle_compute(SHAPE, top_p, rank, n_ranks, placement), placement=placement)
         q.put((rank, out.numpy().copy()))
     finally:
         dist.destroy_process_group()
+
+
+def _usage_placement(n_ranks):
+    # the usage record of the batch's own routing, then its most-used-first order
+    from oracle import oracle as O
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import placement_by_usage
+    x = synth.hidden_states(SHAPE)
+    idx, _, _, _ = O.route(x, synth.router_weight(SHAPE), synth.router_bias(SHAPE), SHAPE.n_group,
+                           SHAPE.topk_group, SHAPE.top_k, SHAPE.rsf)
+    order = O.usage_rank(O.usage_accumulate(idx, SHAPE.E))
+    return placement_by_usage(torch.from_numpy(np.asarray(order)), n_ranks)
 
 
 def _reference(top_p):
@@ -84,13 +100,14 @@ def _reference(top_p):
     return of, idx
 
 
-@pytest.mark.parametrize("top_p", [0.0, 0.6])
-def test_two_ranks_equal_one_process(top_p):
+@pytest.mark.parametrize("top_p,usage_placement", [(0.0, False), (0.6, False), (0.0, True)])
+def test_two_ranks_equal_one_process(top_p, usage_placement):
     splits = [0, 4, SHAPE.T]  # ragged: 4 and 3 tokens
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, top_p, splits, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, top_p, splits, q, usage_placement))
+             for r in range(2)]
     for p in procs:
         p.start()
     try:
@@ -105,8 +122,29 @@ def test_two_ranks_equal_one_process(top_p):
     ref, idx = _reference(top_p)
     if top_p:
         assert (idx < 0).any()  # some slots are empty and go nowhere
-    per = SHAPE.E // 2
-    assert ((idx >= per) & (np.arange(SHAPE.T)[:, None] < 4)).any()  # rank 0 sends to rank 1
-    assert ((idx >= 0) & (idx < per) & (np.arange(SHAPE.T)[:, None] >= 4)).any()  # and back
+    owner = _usage_placement(2)[0].numpy() if usage_placement else np.arange(SHAPE.E) // (SHAPE.E // 2)
+    own = np.where(idx >= 0, owner[np.maximum(idx, 0)], -1)
+    assert ((own == 1) & (np.arange(SHAPE.T)[:, None] < 4)).any()  # rank 0 sends to rank 1
+    assert ((own == 0) & (np.arange(SHAPE.T)[:, None] >= 4)).any()  # and back
     for r in range(2):
         assert np.array_equal(got[r].view(np.uint32), ref[splits[r]:splits[r + 1]].view(np.uint32))
+
+
+def test_placement_by_usage_deals_hot_experts_evenly():
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import experts_of_rank, placement_by_usage
+    rng = np.random.default_rng(3)
+    E, N = 64, 4
+    usage = (1000 * rng.zipf(1.3, E).clip(max=50)).astype(np.int64)
+    order = torch.from_numpy(np.lexsort((np.arange(E), -usage)))  # most used first, ties to the lower index
+    owner, local = placement_by_usage(order, N)
+    held = [experts_of_rank(owner, local, r).numpy() for r in range(N)]
+    assert sorted(np.concatenate(held).tolist()) == list(range(E))  # every expert exactly once
+    assert all(len(h) == E // N for h in held)
+    for r in range(N):  # local indices number each rank's experts in dealing order
+        assert np.array_equal(local.numpy()[held[r]], np.arange(E // N))
+    top = order[:N].numpy()  # the N hottest experts land on N different ranks
+    assert len(set(owner.numpy()[top].tolist())) == N
+    loads = np.array([usage[h].sum() for h in held])
+    contiguous = np.array([usage[r * E // N:(r + 1) * E // N].sum() for r in range(N)])
+    assert loads.max() - loads.min() <= usage.max()  # within one expert's load of even
+    assert loads.max() <= contiguous.max()

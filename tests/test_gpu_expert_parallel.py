@@ -1,7 +1,8 @@
 """Expert parallelism on the GPU: the layer's CUDA compute steps under the
 expert-parallel exchange (one rank: the all-to-alls are local copies), and a
-rank's slice of the experts (rank 1 of 2), against the oracle bit for bit (the
-integer-dot expert kernels fold in the definition's order)."""
+rank's share of the experts (rank 1 of 2, a contiguous slice or dealt by
+usage), against the oracle bit for bit (the integer-dot expert kernels fold
+in the definition's order)."""
 import datetime
 import os
 import socket
@@ -68,4 +69,23 @@ def test_ep_rank_slice_experts():
     y = compute.experts(to_dev_bf16(x), torch.from_numpy(local).cuda()).cpu().numpy()
     routed = oracle_experts(sh, np.unique(local) + per)
     y_o = O.expert_ffn_per_token(routed, x, (local + per).reshape(-1, 1))[:, 0, :]
+    assert np.array_equal(y.view(np.uint32), y_o.view(np.uint32))
+
+
+def test_ep_rank_experts_under_usage_placement():
+    # experts dealt to 2 ranks in a most-used-first order: rank 1 gathers its own stack
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import experts_of_rank, placement_by_usage
+    sh = SHAPES["ep_decode"]
+    dev = device_layer(sh)
+    x, W, b = layer_inputs(sh)
+    idx, _, _, _ = O.route(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf)
+    order = O.usage_rank(O.usage_accumulate(idx, sh.E))
+    placement = placement_by_usage(torch.from_numpy(np.asarray(order)), 2)
+    compute = ep_cuda_compute(dev["W"], dev["bias"], dev["cfg"], dev["routed"], dev["shared"], rank=1, n_ranks=2,
+                              placement=placement)
+    mine = experts_of_rank(*placement, 1).numpy()
+    local = (np.arange(sh.T) * 5 % len(mine)).astype(np.int32)
+    y = compute.experts(to_dev_bf16(x), torch.from_numpy(local).cuda()).cpu().numpy()
+    routed = oracle_experts(sh, np.unique(mine[local]))
+    y_o = O.expert_ffn_per_token(routed, x, mine[local].astype(np.int32).reshape(-1, 1))[:, 0, :]
     assert np.array_equal(y.view(np.uint32), y_o.view(np.uint32))
