@@ -9,20 +9,22 @@
 // blocks in ascending order with one fp32 fused multiply-add per block: the
 // quantised dot of the layer's definition, bit for bit (a one-ulp difference in
 // h could flip a Q8_0 code of h).  The CTA's weight rows pass through shared
-// memory in chunks of kCB blocks, loaded with coalesced 16-byte (int2: 8-byte)
-// reads one chunk ahead in registers: a lane streaming its own row through L1
-// would need more L1 than the SM has beside the staging buffers.  With grouped weight scales ([MO] "int4
-// 양자화 (Quantization)의 품질 비용") block b's factor is d_b * s[g(b)], rounded
-// once, and the row has no separate scale.
+// memory in chunks, loaded with coalesced 16-byte (int2: 8-byte) reads one
+// chunk ahead in registers: a lane streaming its own row through L1 would need
+// more L1 than the SM has beside the staging buffers.  With grouped weight
+// scales ([MO] "int4 양자화 (Quantization)의 품질 비용") block b's factor is
+// d_b * s[g(b)], rounded once, and the row has no separate scale.
 //
-// up/gate kernel: one CTA per (32-row block of h, distinct expert).  It stages
-// the Q8_0 activations of up to kUgTok of the expert's tokens in shared
-// memory; warp w takes the gate (w even) or up (w odd) rows, lane r row r, for
-// the tokens of group w / 2; then SwiGLU and Q8_0 of the 32 h values of each
-// token give one Q8_0 block, written by pair index.
-// down kernel: one CTA per (32 output rows, distinct expert); warp w takes
-// kDownTpw of the expert's staged pairs, lane r output row r; y is written by
-// (token, slot).
+// up/gate kernel: one CTA per (group of h rows, distinct expert).  It stages
+// the Q8_0 activations of a pass's tokens in shared memory; warp w takes the
+// gate (w even) or up (w odd) rows of its 32-row group, lane r row r, for its
+// tokens; then SwiGLU and Q8_0 of each token's 32 h values give one Q8_0 block,
+// written by pair index.
+// down kernel: one CTA per (group of output rows, distinct expert); warp w
+// takes its rows and pairs, lane r output row r; y is written by (token, slot).
+// The CTA geometry (how many rows, how many tokens a pass) is narrow or wide,
+// below.  A shared expert of the routed experts' shape can ride along as grid
+// row 0 of both launches.
 #include <type_traits>
 
 #include "common.cuh"
