@@ -362,9 +362,22 @@ def prefill_measurement(args, moe, L, device_layer, to_dev_bf16):
     }
 
 
+def call_roofline(path: str, call_bytes: float, call_ms: float, kernel_ms: float, hbm: float, kind: str) -> dict:
+    """HBM roofline of one layer call's weight bytes.  On the fused path it is timed per launch of
+    k_decode_fused (the whole layer); on the other paths the profiled region covers only some of
+    the call's launches, so the whole call's time is used."""
+    if path == "fused":
+        ms, kernel, key = kernel_ms, "k_decode_fused", "ms_per_launch"
+    else:
+        ms, kernel, key = call_ms, f"whole layer call ({path} path, several launches)", "ms_per_call"
+    achieved = call_bytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm, "peak_kind": kind,
+            "unit": "GB/s", "frac": achieved / hbm, key: ms}
+
+
 def verify_measurement(moe, L, device_layer, to_dev_bf16, name: str, n_layers: int = 4, steps: int = 200):
-    """MTP verify (T = 4 correlated positions, the fused kernel): tokens/s, the realised batch
-    unions, and the fused kernel's bytes per call against the HBM roofline."""
+    """MTP verify (T = 4 correlated positions; int4 takes the fused kernel, int8 the general path):
+    tokens/s, the realised batch unions, and the call's weight bytes against the HBM roofline."""
     import ctypes
 
     import torch
@@ -417,9 +430,8 @@ def verify_measurement(moe, L, device_layer, to_dev_bf16, name: str, n_layers: i
         "tokens_per_s": T / (ms / 1e3), "ms_per_call": ms,
         "distinct_experts": {"mean": float(U.mean()), "min": int(U.min()), "max": int(U.max())},
         "bytes_per_call": call_bytes, "GBps": call_bytes / (ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "k_decode_fused", "achieved": call_bytes / (k_ms / 1e3) / 1e9,
-                     "peak": hbm, "peak_kind": kind, "unit": "GB/s",
-                     "frac": call_bytes / (k_ms / 1e3) / 1e9 / hbm, "ms_per_launch": k_ms},
+        "roofline": call_roofline({moe.PATH_FUSED: "fused", moe.PATH_TENSOR_CORE: "tensor_core",
+                                   moe.PATH_GENERAL: "general"}[path], call_bytes, ms, k_ms, hbm, kind),
     }
 
 
