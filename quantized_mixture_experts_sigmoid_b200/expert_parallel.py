@@ -45,12 +45,14 @@ class EPCompute:
     route(x) -> (idx [T, K] int32, w [T, K] float32), over all E experts;
     experts(rows, local_idx) -> y [R, H] float32: the rank's experts (local index) on bf16 rows [R, H];
     shared(x) -> y [T, H] float32, or None without a shared expert;
-    combine(y_pairs [T, K, H], w [T, K], shared_y or None) -> out [T, H].
+    combine(y_pairs [T, K, H], w [T, K], shared_y or None) -> out [T, H] of out_dtype.
+    A rank without tokens calls only `experts` (for the rows other ranks send it).
     """
     route: Callable
     experts: Callable
     shared: Optional[Callable]
     combine: Callable
+    out_dtype: torch.dtype = torch.float32
 
 
 def placement_by_usage(order: torch.Tensor, n_ranks: int) -> tuple[torch.Tensor, torch.Tensor]:
@@ -100,9 +102,13 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None,
         raise ValueError(f"{n_expert} experts do not split evenly over {n} ranks")
     per = n_expert // n
     T, H = x.shape
-    idx, w = compute.route(x)
-    K = idx.shape[1]
-    flat = idx.reshape(-1).to(torch.int64)
+    if T:
+        idx, w = compute.route(x)
+        K = idx.shape[1]
+        flat = idx.reshape(-1).to(torch.int64)
+    else:  # no tokens here this call: nothing to send, but this rank's experts still serve the others
+        w, K = None, 1
+        flat = torch.empty(0, dtype=torch.int64, device=x.device)
     valid = flat >= 0
     if placement is None:
         owner_of = torch.where(valid, flat // per, torch.full_like(flat, n))
@@ -123,7 +129,8 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None,
     n_recv = sum(rc)
 
     # the pairs' token rows as raw bf16 bits, two to a 32-bit word (H is even)
-    rows = x.contiguous().view(torch.int32).index_select(0, order // K)
+    rows = (x.contiguous().view(torch.int32).index_select(0, order // K) if n_send
+            else torch.empty(0, H // 2, dtype=torch.int32, device=x.device))
     local = local_of[order].to(torch.int32)  # expert index on the destination rank
     recv_rows = _a2a(torch.empty(n_recv, H // 2, dtype=torch.int32, device=x.device), rows, rc, sc, group)
     recv_local = _a2a(torch.empty(n_recv, dtype=torch.int32, device=x.device), local, rc, sc, group)
@@ -131,6 +138,8 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None,
     y_recv = compute.experts(recv_rows.view(torch.bfloat16), recv_local) if n_recv else \
         torch.empty(0, H, dtype=torch.float32, device=x.device)
     y_back = _a2a(torch.empty(n_send, H, dtype=torch.float32, device=x.device), y_recv.contiguous(), sc, rc, group)
+    if not T:
+        return torch.empty(0, H, dtype=compute.out_dtype, device=x.device)
 
     y_pairs = torch.zeros(T * K, H, dtype=torch.float32, device=x.device)
     y_pairs.index_copy_(0, order, y_back)
@@ -203,4 +212,4 @@ def ep_cuda_compute(w_router: torch.Tensor, bias: torch.Tensor, cfg, routed, sha
         moe.moe_combine(y_pairs, w, shared_y, out)
         return out
 
-    return EPCompute(route, experts, shared_fn if shared is not None else None, combine)
+    return EPCompute(route, experts, shared_fn if shared is not None else None, combine, out_dtype)

@@ -100,9 +100,11 @@ def _reference(top_p):
     return of, idx
 
 
-@pytest.mark.parametrize("top_p,usage_placement", [(0.0, False), (0.6, False), (0.0, True)])
-def test_two_ranks_equal_one_process(top_p, usage_placement):
-    splits = [0, 4, SHAPE.T]  # ragged: 4 and 3 tokens
+@pytest.mark.parametrize("top_p,usage_placement,split", [(0.0, False, 4), (0.6, False, 4), (0.0, True, 4),
+                                                         (0.0, False, SHAPE.T)])
+def test_two_ranks_equal_one_process(top_p, usage_placement, split):
+    # ragged: 4 and 3 tokens; or rank 1 without tokens (it still serves its experts)
+    splits = [0, split, SHAPE.T]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _port()
@@ -124,8 +126,9 @@ def test_two_ranks_equal_one_process(top_p, usage_placement):
         assert (idx < 0).any()  # some slots are empty and go nowhere
     owner = _usage_placement(2)[0].numpy() if usage_placement else np.arange(SHAPE.E) // (SHAPE.E // 2)
     own = np.where(idx >= 0, owner[np.maximum(idx, 0)], -1)
-    assert ((own == 1) & (np.arange(SHAPE.T)[:, None] < 4)).any()  # rank 0 sends to rank 1
-    assert ((own == 0) & (np.arange(SHAPE.T)[:, None] >= 4)).any()  # and back
+    assert ((own == 1) & (np.arange(SHAPE.T)[:, None] < split)).any()  # rank 0 sends to rank 1
+    if split < SHAPE.T:
+        assert ((own == 0) & (np.arange(SHAPE.T)[:, None] >= split)).any()  # and back
     for r in range(2):
         assert np.array_equal(got[r].view(np.uint32), ref[splits[r]:splits[r + 1]].view(np.uint32))
 
