@@ -88,6 +88,29 @@ def _usage_placement(n_ranks):
     return placement_by_usage(torch.from_numpy(np.asarray(order)), n_ranks)
 
 
+def test_four_ranks_equal_one_process():
+    # every rank sends to and receives from several others; ranks of 2, 1, 0 and 4 tokens
+    splits = [0, 2, 3, 3, SHAPE.T]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 4, port, 0.0, splits, q, True)) for r in range(4)]
+    for p in procs:
+        p.start()
+    try:
+        got = dict(q.get(timeout=90) for _ in procs)
+        for p in procs:
+            p.join(timeout=60)
+            assert p.exitcode == 0
+    finally:
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+    ref, _ = _reference(0.0)
+    for r in range(4):
+        assert np.array_equal(got[r].view(np.uint32), ref[splits[r]:splits[r + 1]].view(np.uint32))
+
+
 def _reference(top_p):
     from oracle import oracle as O
     from oracle.synth_inputs import oracle_experts
