@@ -8,8 +8,8 @@ the router and of the shared expert, and its own tokens.  One call:
 
 1. routes the rank's tokens (every rank routes over all E experts);
 2. sends each (token, slot) pair's token row to the rank holding the pair's
-   expert (all-to-all, rows as raw bf16 bits in 32-bit words) with the
-   expert's local index;
+   expert with the expert's local index (one all-to-all of 32-bit words: the
+   row's raw bf16 bits, then the index);
 3. runs the rank's experts over the rows it received (a batch union over the
    local experts, then the quantised SwiGLU experts);
 4. returns every pair's expert output to the token's rank (all-to-all);
@@ -128,15 +128,17 @@ def ep_forward(x: torch.Tensor, n_expert: int, compute: EPCompute, group=None,
     sc, rc = send_counts.tolist(), recv_counts.tolist()
     n_recv = sum(rc)
 
-    # the pairs' token rows as raw bf16 bits, two to a 32-bit word (H is even)
-    rows = (x.contiguous().view(torch.int32).index_select(0, order // K) if n_send
-            else torch.empty(0, H // 2, dtype=torch.int32, device=x.device))
-    local = local_of[order].to(torch.int32)  # expert index on the destination rank
-    recv_rows = _a2a(torch.empty(n_recv, H // 2, dtype=torch.int32, device=x.device), rows, rc, sc, group)
-    recv_local = _a2a(torch.empty(n_recv, dtype=torch.int32, device=x.device), local, rc, sc, group)
+    # one message per pair: the token row as raw bf16 bits, two to a 32-bit word (H is even), then
+    # the expert's index on the destination rank
+    W = H // 2
+    send = torch.empty(n_send, W + 1, dtype=torch.int32, device=x.device)
+    if n_send:
+        send[:, :W] = x.contiguous().view(torch.int32).index_select(0, order // K)
+        send[:, W] = local_of[order].to(torch.int32)
+    recv = _a2a(torch.empty(n_recv, W + 1, dtype=torch.int32, device=x.device), send, rc, sc, group)
 
-    y_recv = compute.experts(recv_rows.view(torch.bfloat16), recv_local) if n_recv else \
-        torch.empty(0, H, dtype=torch.float32, device=x.device)
+    y_recv = compute.experts(recv[:, :W].contiguous().view(torch.bfloat16), recv[:, W].contiguous()) if n_recv \
+        else torch.empty(0, H, dtype=torch.float32, device=x.device)
     y_back = _a2a(torch.empty(n_send, H, dtype=torch.float32, device=x.device), y_recv.contiguous(), sc, rc, group)
     if not T:
         return torch.empty(0, H, dtype=compute.out_dtype, device=x.device)
