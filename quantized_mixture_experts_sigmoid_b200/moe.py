@@ -4,6 +4,12 @@ Every step of the layer runs in the library's CUDA kernels.  Tensors are
 passed as device pointers (``tensor.data_ptr()``) together with the current
 torch CUDA stream; torch supplies device memory and streams, nothing else.
 There is no CPU fallback: if the library cannot be loaded, every call raises.
+
+The library sees only addresses and sizes, so the binding checks what it
+cannot before passing a tensor: that it lives on a CUDA device, is
+contiguous, has elements of the width the C signature reads, and holds at
+least the elements the call will touch (a host tensor or a short buffer would
+otherwise be read or written out of bounds on the device).
 """
 from __future__ import annotations
 
@@ -48,9 +54,13 @@ class _Experts(ctypes.Structure):
                 ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p), ("group_size", ctypes.c_int)]
 
 
-@dataclass
+@dataclass(frozen=True)
 class ExpertSet:
     """A stack of experts resident on the device (tensors owned by the caller).
+
+    Checked once when made (device, contiguity, element widths, sizes); its C struct is built
+    then too, so a layer call only passes it.  Fields cannot be reassigned (the tensors' contents
+    can change in place).
 
     w_gate, w_up: uint8 [n, inter, hidden*q/8]; w_down: uint8 [n, hidden, inter*q/8];
     s_gate, s_up: fp32 [n, inter]; s_down: fp32 [n, hidden]; with grouped scales (group_size G)
@@ -68,10 +78,20 @@ class ExpertSet:
     s_down: torch.Tensor
     group_size: int = 0
 
+    def __post_init__(self):
+        q, n, H, I, G = self.qtype, self.n_expert, self.hidden, self.inter, self.group_size
+        per_h = H // G if G > 0 else 1
+        per_i = I // G if G > 0 else 1
+        for name, width, count in (("w_gate", 1, n * I * H * q // 8), ("w_up", 1, n * I * H * q // 8),
+                                   ("w_down", 1, n * H * I * q // 8), ("s_gate", 4, n * I * per_h),
+                                   ("s_up", 4, n * I * per_h), ("s_down", 4, n * H * per_i)):
+            _dev(getattr(self, name), width, count, name)
+        object.__setattr__(self, "_struct", _Experts(
+            q, n, H, I, self.w_gate.data_ptr(), self.w_up.data_ptr(), self.w_down.data_ptr(),
+            self.s_gate.data_ptr(), self.s_up.data_ptr(), self.s_down.data_ptr(), G))
+
     def struct(self) -> _Experts:
-        return _Experts(self.qtype, self.n_expert, self.hidden, self.inter, self.w_gate.data_ptr(),
-                        self.w_up.data_ptr(), self.w_down.data_ptr(), self.s_gate.data_ptr(),
-                        self.s_up.data_ptr(), self.s_down.data_ptr(), self.group_size)
+        return self._struct
 
     @staticmethod
     def empty(qtype: int, n_expert: int, hidden: int, inter: int, device="cuda", group_size: int = 0) -> "ExpertSet":
@@ -142,8 +162,26 @@ def strerror(code: int) -> str:
     return lib().moe_strerror(int(code)).decode()
 
 
-def _ptr(t):
-    return None if t is None else t.data_ptr()
+def _dev(t, width: int, count: int, name: str):
+    """t's device address once t is a contiguous CUDA tensor of `width`-byte elements holding at
+    least `count` of them; None (an optional argument) stays None."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name}: a CUDA tensor is required, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.element_size() != width:
+        raise TypeError(f"{name}: elements of {width} bytes expected, got {t.dtype}")
+    if t.numel() < count:
+        raise ValueError(f"{name}: {count} elements needed, {t.numel()} given")
+    return t.data_ptr()
+
+
+def _ws(ws):
+    """A workspace's address and size in bytes."""
+    _dev(ws, ws.element_size(), 0, "ws")
+    return ws.data_ptr(), ws.numel() * ws.element_size()
 
 
 def _stream(stream):
@@ -168,34 +206,39 @@ def moe_route_workspace_bytes(T: int, cfg: RouterCfg) -> int:
     return lib().moe_route_workspace_bytes(T, ctypes.byref(cfg))
 
 
-def moe_route(x, w_router, bias, cfg: RouterCfg, topk_idx, topk_w, ws, stream=None):
+def _route_args(x, w_router, bias, cfg, topk_idx, topk_w):
     T, H = x.shape
-    _ok("moe_route", lib().moe_route(_ptr(x), T, H, _ptr(w_router), _ptr(bias), ctypes.byref(cfg),
-                                     _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
+    E, K = cfg.n_expert, cfg.top_k
+    return (_dev(x, 2, T * H, "x"), T, H, _dev(w_router, 4, E * H, "w_router"), _dev(bias, 4, E, "bias"),
+            ctypes.byref(cfg), _dev(topk_idx, 4, T * K, "topk_idx"), _dev(topk_w, 4, T * K, "topk_w"))
+
+
+def moe_route(x, w_router, bias, cfg: RouterCfg, topk_idx, topk_w, ws, stream=None):
+    _ok("moe_route", lib().moe_route(*_route_args(x, w_router, bias, cfg, topk_idx, topk_w), *_ws(ws),
                                      _stream(stream)))
 
 
 def moe_route_noalloc(x, w_router, bias, cfg: RouterCfg, topk_idx, topk_w, stream=None):
     """moe_route with the library's built-in logits scratch (no workspace, allocates nothing)."""
-    T, H = x.shape
-    _ok("moe_route_noalloc", lib().moe_route_noalloc(_ptr(x), T, H, _ptr(w_router), _ptr(bias),
-                                                     ctypes.byref(cfg), _ptr(topk_idx),
-                                                     _ptr(topk_w), _stream(stream)))
+    _ok("moe_route_noalloc", lib().moe_route_noalloc(*_route_args(x, w_router, bias, cfg, topk_idx, topk_w),
+                                                     _stream(stream)))
 
 
 def moe_union(topk_idx, E, n_unique, uniq, offsets, pair_tok, pair_slot, counts=None,
               status=None, stream=None):
     T, K = topk_idx.shape
-    _ok("moe_union", lib().moe_union(_ptr(topk_idx), T, K, E, _ptr(n_unique), _ptr(uniq),
-                                     _ptr(offsets), _ptr(pair_tok), _ptr(pair_slot), _ptr(counts),
-                                     _ptr(status), _stream(stream)))
+    _ok("moe_union", lib().moe_union(_dev(topk_idx, 4, T * K, "topk_idx"), T, K, E, _dev(n_unique, 4, 1, "n_unique"),
+                                     _dev(uniq, 4, E, "uniq"), _dev(offsets, 4, E + 1, "offsets"),
+                                     _dev(pair_tok, 4, T * K, "pair_tok"), _dev(pair_slot, 4, T * K, "pair_slot"),
+                                     _dev(counts, 4, E, "counts"), _dev(status, 4, 1, "status"), _stream(stream)))
 
 
 def moe_quantize_q8_0(v, q, d, stream=None):
     rows, n = v.shape
     dt = MOE_OUT_BF16 if v.dtype in (torch.bfloat16, torch.int16, torch.uint16) else MOE_OUT_F32
-    _ok("moe_quantize_q8_0", lib().moe_quantize_q8_0(_ptr(v), dt, rows, n, _ptr(q), _ptr(d),
-                                                     _stream(stream)))
+    _ok("moe_quantize_q8_0", lib().moe_quantize_q8_0(_dev(v, 2 if dt == MOE_OUT_BF16 else 4, rows * n, "v"), dt,
+                                                     rows, n, _dev(q, 1, rows * n, "q"),
+                                                     _dev(d, 4, rows * (n // 32), "d"), _stream(stream)))
 
 
 def moe_expert_ffn_workspace_bytes(ex: ExpertSet, T: int, top_k: int) -> int:
@@ -207,17 +250,23 @@ def moe_expert_ffn_q(ex: ExpertSet, x, top_k, union, y_pairs, ws, stream=None):
     """union: (n_unique, uniq, offsets, pair_tok, pair_slot) device tensors, or None (dense)."""
     T = x.shape[0]
     s = ex.struct()
-    u = (None,) * 5 if union is None else union
-    _ok("moe_expert_ffn_q", lib().moe_expert_ffn_q(ctypes.byref(s), _ptr(x), T, top_k,
-                                                   *[_ptr(a) for a in u], _ptr(y_pairs), _ptr(ws),
-                                                   ws.numel(), _stream(stream)))
+    if union is None:
+        u = (None,) * 5
+    else:
+        nu, uq, of, pt, ps = union
+        u = (_dev(nu, 4, 1, "n_unique"), _dev(uq, 4, 0, "uniq"), _dev(of, 4, 1, "offsets"),
+             _dev(pt, 4, T * top_k, "pair_tok"), _dev(ps, 4, T * top_k, "pair_slot"))
+    _ok("moe_expert_ffn_q", lib().moe_expert_ffn_q(ctypes.byref(s), _dev(x, 2, T * ex.hidden, "x"), T, top_k, *u,
+                                                   _dev(y_pairs, 4, T * top_k * ex.hidden, "y_pairs"), *_ws(ws),
+                                                   _stream(stream)))
 
 
 def moe_combine(y_pairs, topk_w, shared_y, out, stream=None):
     T, K, H = y_pairs.shape
     dt = MOE_OUT_F32 if out.dtype == torch.float32 else MOE_OUT_BF16
-    _ok("moe_combine", lib().moe_combine(_ptr(y_pairs), _ptr(topk_w), _ptr(shared_y), T, K, H,
-                                         _ptr(out), dt, _stream(stream)))
+    _ok("moe_combine", lib().moe_combine(_dev(y_pairs, 4, T * K * H, "y_pairs"), _dev(topk_w, 4, T * K, "topk_w"),
+                                         _dev(shared_y, 4, T * H, "shared_y"), T, K, H,
+                                         _dev(out, 4 if dt == MOE_OUT_F32 else 2, T * H, "out"), dt, _stream(stream)))
 
 
 def moe_layer_workspace_bytes(T: int, cfg: RouterCfg, routed: ExpertSet, shared: ExpertSet | None):
@@ -243,33 +292,38 @@ def moe_layer_path(T: int, cfg: RouterCfg, routed: ExpertSet, shared: ExpertSet 
 def moe_layer_forward(x, w_router, bias, cfg: RouterCfg, routed: ExpertSet,
                       shared: ExpertSet | None, out, ws, topk_idx=None, topk_w=None, stream=None):
     T = x.shape[0]
+    H, E, K = routed.hidden, cfg.n_expert, cfg.top_k
     rs = routed.struct()
     ss = shared.struct() if shared is not None else None
     dt = MOE_OUT_F32 if out.dtype == torch.float32 else MOE_OUT_BF16
     _ok("moe_layer_forward", lib().moe_layer_forward(
-        _ptr(x), T, _ptr(w_router), _ptr(bias), ctypes.byref(cfg), ctypes.byref(rs),
-        ctypes.byref(ss) if ss is not None else None, _ptr(out), dt, _ptr(topk_idx), _ptr(topk_w),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        _dev(x, 2, T * H, "x"), T, _dev(w_router, 4, E * H, "w_router"), _dev(bias, 4, E, "bias"), ctypes.byref(cfg),
+        ctypes.byref(rs), ctypes.byref(ss) if ss is not None else None,
+        _dev(out, 4 if dt == MOE_OUT_F32 else 2, T * H, "out"), dt, _dev(topk_idx, 4, T * K, "topk_idx"),
+        _dev(topk_w, 4, T * K, "topk_w"), *_ws(ws), _stream(stream)))
 
 
 def moe_usage_accumulate(topk_idx, E: int, usage, stream=None) -> None:
     """usage[e] += entries of topk_idx [T][K] routed to e (empty slots add nothing)."""
     T, K = topk_idx.shape
-    _ok("moe_usage_accumulate", lib().moe_usage_accumulate(_ptr(topk_idx), T, K, int(E), _ptr(usage), _stream(stream)))
+    _ok("moe_usage_accumulate", lib().moe_usage_accumulate(_dev(topk_idx, 4, T * K, "topk_idx"), T, K, int(E),
+                                                           _dev(usage, 4, int(E), "usage"), _stream(stream)))
 
 
 def moe_usage_rank(usage, order, stream=None) -> None:
     """order[r] = the expert of rank r in the usage record (most used first, ties to the lower index)."""
-    _ok("moe_usage_rank", lib().moe_usage_rank(_ptr(usage), usage.numel(), _ptr(order), _stream(stream)))
+    E = usage.numel()
+    _ok("moe_usage_rank", lib().moe_usage_rank(_dev(usage, 4, E, "usage"), E, _dev(order, 4, E, "order"),
+                                               _stream(stream)))
 
 
 def moe_workspace_set_wait_limit(ws, polls: int, stream=None) -> None:
     """Test knob: cap every bounded device wait of later calls on `ws` at `polls` polls (0: defaults)."""
-    _ok("moe_workspace_set_wait_limit", lib().moe_workspace_set_wait_limit(_ptr(ws), int(polls), _stream(stream)))
+    _ok("moe_workspace_set_wait_limit", lib().moe_workspace_set_wait_limit(_ws(ws)[0], int(polls), _stream(stream)))
 
 
 def moe_workspace_status(ws, clear: bool = True, stream=None) -> int:
     st = ctypes.c_int(0)
-    _ok("moe_workspace_status", lib().moe_workspace_status(_ptr(ws), int(clear), ctypes.byref(st),
+    _ok("moe_workspace_status", lib().moe_workspace_status(_ws(ws)[0], int(clear), ctypes.byref(st),
                                                            _stream(stream)))
     return st.value
