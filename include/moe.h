@@ -197,9 +197,10 @@ int moe_route_noalloc(const uint16_t* x, int T, int H, const float* w_router, co
  *   counts (optional, NULL)   [E] entries per expert (all E, zeros included)
  * Entries of uniq / offsets past U are left unspecified.  An index of -1 is
  * an empty slot (dropped by top-p, or a token the router could not route)
- * and has no pair; any other index outside [0, E) is skipped too and recorded
- * as MOE_EDEVICE_INDEX in `status` (optional device int32, not cleared by
- * this call).  The offsets[U] valid pairs come first in pair_tok / pair_slot;
+ * and has no pair; any other index outside [0, E), and any repeat of an
+ * expert earlier in the same row, is skipped too and recorded as
+ * MOE_EDEVICE_INDEX in `status` (optional device int32, not cleared by this
+ * call).  The offsets[U] valid pairs come first in pair_tok / pair_slot;
  * the remaining entries of the T*top_k get token 0 and slot -1.  One CTA; no
  * workspace.
  */

@@ -8,7 +8,10 @@
 //
 // An index of -1 is an empty slot (dropped by adaptive top-p, or a token the
 // router could not route): it has no pair.  Any other index outside [0, E)
-// records MOE_EDEVICE_INDEX and is left out too.  The pair lists hold the
+// records MOE_EDEVICE_INDEX and is left out too, and so is a repeat of an
+// expert earlier in the same row (rows must be distinct; a repeat would
+// otherwise take the same pair position as its first entry and leave a hole in
+// the lists, which later kernels would read as a token).  The pair lists hold the
 // valid pairs first (offsets[n_unique] of them); the rest of the T*K entries
 // get token 0, slot -1, so a pass that walks all T*K rows reads valid rows.
 //
@@ -35,6 +38,13 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
     return v;
 }
 
+// Whether entry k of a row of top_k indices repeats an earlier entry of the row.
+__device__ __forceinline__ bool repeats_earlier(const int32_t* __restrict__ row, int k, int e) {
+    for (int j = 0; j < k; ++j)
+        if (row[j] == e) return true;
+    return false;
+}
+
 __global__ void __launch_bounds__(kUnionThreads)
 k_union(const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restrict__ n_unique,
         int32_t* __restrict__ uniq, int32_t* __restrict__ offsets, int32_t* __restrict__ pair_tok,
@@ -51,7 +61,9 @@ k_union(const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restric
     const long n = static_cast<long>(T) * K;
     for (long i = tid; i < n; i += kUnionThreads) {
         const int e = idx[i];
-        if (e >= 0 && e < E) {
+        const long t = i / K;
+        const int k = static_cast<int>(i - t * K);
+        if (e >= 0 && e < E && !repeats_earlier(idx + t * K, k, e)) {
             atomicAdd(&cnt[e], 1);
         } else if (e != -1) {
             record_status(status, MOE_EDEVICE_INDEX);
@@ -119,7 +131,7 @@ k_union(const int32_t* __restrict__ idx, int T, int K, int E, int32_t* __restric
         if (t < T) {
             for (int k = 0; k < K; ++k) {
                 const int e = idx[static_cast<size_t>(t) * K + k];
-                if (e < 0 || e >= E) continue;
+                if (e < 0 || e >= E || repeats_earlier(idx + static_cast<size_t>(t) * K, k, e)) continue;
                 const uint32_t* row = bm + e * kChunkWords;
                 int rank = __popc(row[warp] & (mybit - 1u));
                 for (int w = 0; w < warp; ++w) rank += __popc(row[w]);

@@ -155,6 +155,33 @@ def test_union_all_tokens_same_experts_and_bad_index():
     assert g["status"] == moe.MOE_EDEVICE_INDEX
 
 
+def test_union_leaves_out_a_repeated_expert():
+    # a malformed row (one expert twice) is recorded and its repeat dropped; the pair lists
+    # stay gap-free (equal to the lists of the same rows with the repeats emptied)
+    rng = np.random.default_rng(5)
+    T, E, K = 300, 64, 6
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[7, 4] = idx[7, 1]
+    idx[250, 5] = idx[250, 0]
+    idx[299, 2] = idx[299, 3] = idx[299, 1]
+    emptied = idx.copy()
+    for t in range(T):
+        for k in range(K):
+            if idx[t, k] in idx[t, :k]:
+                emptied[t, k] = -1
+    assert (emptied == -1).sum() == 4
+    g, o = gpu_union(idx, E), O.union(emptied, E)
+    n = int(o["offsets"][o["n_unique"]])
+    assert g["status"] == moe.MOE_EDEVICE_INDEX and n == T * K - 4
+    assert g["n_unique"] == o["n_unique"]
+    assert np.array_equal(g["uniq"], o["uniq"][:o["n_unique"]])
+    assert np.array_equal(g["offsets"], o["offsets"][:o["n_unique"] + 1])
+    assert np.array_equal(g["counts"], o["counts"])
+    assert np.array_equal(g["pair_tok"][:n], o["pair_tok"][:n])
+    assert np.array_equal(g["pair_slot"][:n], o["pair_slot"][:n])
+    assert np.all(g["pair_tok"][n:] == 0) and np.all(g["pair_slot"][n:] == -1)
+
+
 # ------------------------------------------------------------------- Q8_0
 @pytest.mark.parametrize("n", [32, 544, 6144])
 def test_q8_0_bit_exact(n):
