@@ -69,6 +69,15 @@ int oracle_route(const uint16_t* x, int T, int H, const float* w_router, const f
                  int E, int n_group, int topk_group, int top_k, float rsf, int32_t* topk_idx,
                  float* topk_w, float* gap_expert, float* gap_group);
 
+/* The same with adaptive expert top-p (0 < top_p < 1; any other value: as above). */
+int oracle_select_topp(const float* logits, int T, const float* bias, int E, int n_group,
+                       int topk_group, int top_k, float rsf, float top_p, int32_t* topk_idx,
+                       float* topk_w, float* gap_expert, float* gap_group);
+
+int oracle_route_topp(const uint16_t* x, int T, int H, const float* w_router, const float* bias,
+                      int E, int n_group, int topk_group, int top_k, float rsf, float top_p,
+                      int32_t* topk_idx, float* topk_w, float* gap_expert, float* gap_group);
+
 int oracle_union(const int32_t* topk_idx, int T, int top_k, int E, int32_t* n_unique,
                  int32_t* uniq, int32_t* offsets, int32_t* pair_tok, int32_t* pair_slot,
                  int32_t* counts);
@@ -98,6 +107,11 @@ int oracle_layer_forward(const uint16_t* x, int T, const float* w_router, const 
                          int E, int n_group, int topk_group, int top_k, float rsf,
                          const oracle_experts* routed, const oracle_experts* shared,
                          float* out_f32, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w);
+
+int oracle_layer_forward_topp(const uint16_t* x, int T, const float* w_router, const float* bias,
+                              int E, int n_group, int topk_group, int top_k, float rsf, float top_p,
+                              const oracle_experts* routed, const oracle_experts* shared,
+                              float* out_f32, uint16_t* out_bf16, int32_t* topk_idx, float* topk_w);
 
 #ifdef __cplusplus
 }
