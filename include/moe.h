@@ -261,8 +261,12 @@ size_t moe_expert_ffn_workspace_bytes(const moe_experts* ex, int T, int top_k);
  * fp32 accumulator starting at 0 that takes one fused multiply-add per block
  * in ascending b, then one fp32 multiply by the row scale; silu(g) =
  * g / (1 + e^-g) is evaluated in fp64 and rounded once to fp32, and h is the
- * fp32 product silu(g) * u.
- * and y_pairs[t][slot][:] = y for each pair (t, slot) of the expert.
+ * fp32 product silu(g) * u; y_pairs[t][slot][:] = y for each pair (t, slot)
+ * of the expert.  The five union arrays are device memory laid out as
+ * moe_union writes them for a topk_idx of the same T and top_k; their entries
+ * are not range-checked on the device (a token outside [0, T), a slot outside
+ * [0, top_k) or an expert outside [0, n_expert) would be read or written out
+ * of bounds), so pass lists that moe_union built.
  * Pass n_unique = uniq = offsets = pair_tok = pair_slot = NULL to apply expert
  * 0 of `ex` to every token (the shared expert); top_k must then be 1.
  * x: [T][H] bf16; y_pairs: [T][top_k][H] fp32 out (entries of pairs that are
