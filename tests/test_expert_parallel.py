@@ -174,3 +174,33 @@ def test_placement_by_usage_deals_hot_experts_evenly():
     contiguous = np.array([usage[r * E // N:(r + 1) * E // N].sum() for r in range(N)])
     assert loads.max() - loads.min() <= usage.max()  # within one expert's load of even
     assert loads.max() <= contiguous.max()
+
+
+def test_placement_by_usage_properties_hold_for_any_usage():
+    # for any usage record and rank count: each rank holds E / N experts numbered 0 .. E/N - 1 in
+    # dealing order, the N hottest sit on N different ranks, and two ranks' loads differ by at most
+    # the largest single expert's usage (snake dealing of a sorted list)
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    from quantized_mixture_experts_sigmoid_b200.expert_parallel import experts_of_rank, placement_by_usage
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.integers(1, 8).flatmap(lambda n: st.tuples(
+        st.just(n), st.lists(st.integers(0, 10**6), min_size=n, max_size=16 * n).map(lambda u: u[:len(u) // n * n]))))
+    def check(case):
+        N, usage = case
+        usage = np.array(usage, dtype=np.int64)
+        E = len(usage)
+        order = torch.from_numpy(np.lexsort((np.arange(E), -usage)))
+        owner, local = placement_by_usage(order, N)
+        held = [experts_of_rank(owner, local, r).numpy() for r in range(N)]
+        assert sorted(np.concatenate(held).tolist()) == list(range(E))
+        for r in range(N):
+            assert len(held[r]) == E // N
+            assert np.array_equal(local.numpy()[held[r]], np.arange(E // N))
+        assert len(set(owner.numpy()[order[:N].numpy()].tolist())) == N
+        loads = np.array([usage[h].sum() for h in held])
+        assert loads.max() - loads.min() <= usage.max()
+
+    check()
