@@ -11,8 +11,8 @@ import torch
 
 import synth
 from oracle import oracle as O
+from synth.device import bits, device_layer, to_dev_bf16
 from tests.helpers import layer_inputs, oracle_experts, rel_err_rows
-from tests.gpu_fixtures import bits, device_layer, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 

@@ -17,7 +17,7 @@ import synth
 from oracle import oracle as O
 from oracle.variant_report import layer_outputs
 from quantized_mixture_experts_sigmoid_b200 import moe
-from tests.gpu_fixtures import device_layer, to_dev_bf16
+from synth.device import device_layer, to_dev_bf16
 from tests.helpers import rel_err_rows
 
 pytestmark = pytest.mark.gpu

@@ -10,7 +10,7 @@ import torch
 import synth
 from oracle import oracle as O
 from quantized_mixture_experts_sigmoid_b200 import moe
-from tests.gpu_fixtures import bits, to_dev_bf16
+from synth.device import bits, to_dev_bf16
 from tests.helpers import layer_inputs, oracle_experts, rel_err_rows
 from tests.test_gpu_parity import TOL, gpu_union, layer
 

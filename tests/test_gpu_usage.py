@@ -8,7 +8,7 @@ import torch
 import synth
 from oracle import oracle as O
 from quantized_mixture_experts_sigmoid_b200 import moe
-from synth.device import device_layer, to_dev_bf16
+from synth.device import to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 

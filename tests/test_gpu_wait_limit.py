@@ -12,7 +12,7 @@ import torch
 
 import synth
 from quantized_mixture_experts_sigmoid_b200 import moe
-from tests.gpu_fixtures import bits, device_layer, to_dev_bf16
+from synth.device import bits, device_layer, to_dev_bf16
 from tests.helpers import layer_inputs
 
 pytestmark = pytest.mark.gpu

@@ -15,7 +15,7 @@ import torch
 
 import synth
 from quantized_mixture_experts_sigmoid_b200 import moe
-from tests.gpu_fixtures import to_dev_bf16
+from synth.device import to_dev_bf16
 
 
 def _route_both(sh, tokens):
