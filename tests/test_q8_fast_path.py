@@ -17,11 +17,11 @@ def _codes(v):
     keep = d[:, 0] != 0
     v, d = v[keep], d[keep]
     exact = np.clip(_round_away((v / d).astype(np.float32).astype(np.float64)), -127, 127)
-    with np.errstate(over="ignore", invalid="ignore"):
+    with np.errstate(over="ignore", invalid="ignore"):  # 1/d may overflow: t is then inf and divides
         r = (np.float32(1) / d).astype(np.float32)
         t = (v * r).astype(np.float32)
-    a = np.abs(t)
-    fast_ok = (a <= 128) & (np.abs(a - np.floor(a) - np.float32(0.5)) >= np.float32(1e-4))
+        a = np.abs(t)
+        fast_ok = (a <= 128) & (np.abs(a - np.floor(a) - np.float32(0.5)) >= np.float32(1e-4))
     fast = np.clip(_round_away(np.where(fast_ok, t, 0).astype(np.float64)), -127, 127)
     shortcut = np.where(fast_ok, fast, exact)
     return exact, shortcut, fast_ok
