@@ -1,9 +1,12 @@
 """Python marshalling for the CPU oracle (liboracle.so) -- TEST INFRASTRUCTURE ONLY.
 
 Only tests/, the package smoke check and bench.py's CPU-baseline leg may
-import this module.  The GPU library never loads it, and this file contains no
+import this module.  The GPU library never loads it.  This file contains no
 arithmetic of the layer: it builds the C library, converts numpy arrays into
-pointers and calls the C functions of moe_oracle.c.
+pointers and calls the C functions of moe_oracle.c.  The one exception is the
+expert-usage record at the end: two plain definitions (count the routed
+entries per expert; order the experts by count), written in Python because
+they involve no floating point.
 """
 from __future__ import annotations
 
