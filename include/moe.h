@@ -108,8 +108,8 @@ typedef struct {
  * [n_expert][inter][hidden/G]; s_down: [n_expert][hidden][inter/G].  Block b
  * of a row then takes the factor d_b * s[g(b)] (rounded once to fp32) in the
  * fold of the quantised dot and the row has no separate scale.  Batches above
- * the fused kernel's size take the general path with grouped scales (the
- * tensor-core path reports MOE_PATH_GENERAL for them). */
+ * the fused kernel's size take the general path with grouped scales, never the
+ * tensor-core path (moe_layer_path reports MOE_PATH_GENERAL for them). */
 typedef struct {
     int qtype;
     int n_expert;
@@ -121,7 +121,7 @@ typedef struct {
     const float* s_gate;
     const float* s_up;
     const float* s_down;
-    int group_size;  /* 0: per-row scales as above; else grouped scales (see below) */
+    int group_size;  /* 0: per-row scales; else grouped scales of group_size codes (above) */
 } moe_experts;
 
 /* ------------------------------------------------------------------ route */
