@@ -1,8 +1,9 @@
-"""Expert parallelism across ranks (the routed experts split by expert, one
-all-to-all each way): two gloo ranks on the CPU, each with its own tokens and
-half of the experts, the compute steps given by the oracle; every rank's
-output rows equal the single-process oracle layer's bit for bit, with and
-without adaptive top-p (empty slots are not sent).
+"""Expert parallelism across ranks (the routed experts split by expert; after
+the counts, one all-to-all each way): two or four gloo ranks on the CPU, each
+with its own tokens (a rank may have none) and its share of the experts, the
+compute steps given by the oracle; every rank's output rows equal the
+single-process oracle layer's bit for bit, with and without adaptive top-p
+(empty slots are not sent), under contiguous and usage-dealt placements.
 """
 import os
 import socket
