@@ -293,7 +293,10 @@ int moe_combine(const float* y_pairs, const float* topk_w, const float* shared_y
 
 /* ------------------------------------------------------------------ layer */
 
-/* Bytes of workspace moe_layer_forward needs. */
+/* Bytes of workspace moe_layer_forward needs (a multiple of 256); 0 for a bad
+ * router configuration or T < 0.  Only the shape fields of the expert structs
+ * are read (not their pointers), so the size can be queried before the
+ * weights exist; moe_layer_forward checks the rest. */
 size_t moe_layer_workspace_bytes(int T, const moe_router_cfg* cfg, const moe_experts* routed,
                                  const moe_experts* shared);
 
