@@ -54,7 +54,7 @@ class _Experts(ctypes.Structure):
                 ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p), ("group_size", ctypes.c_int)]
 
 
-@dataclass(frozen=True)
+@dataclass(frozen=True, eq=False)  # compared and hashed by identity: the fields are device tensors
 class ExpertSet:
     """A stack of experts resident on the device (tensors owned by the caller).
 
