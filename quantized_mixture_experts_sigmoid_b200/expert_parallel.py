@@ -27,7 +27,9 @@ hot ones and of the routed pairs.
 
 The exchange is plain collectives (NCCL between GPUs); the compute steps are
 this library's C-ABI calls (`ep_cuda_compute`) or, in tests, any functions of
-the same signatures.
+the same signatures.  Device-side errors that the kernels record (a bounded
+wait that gave up, an index out of range) are read after a call with the
+compute's `status()`.
 """
 from __future__ import annotations
 
@@ -47,12 +49,15 @@ class EPCompute:
     shared(x) -> y [T, H] float32, or None without a shared expert;
     combine(y_pairs [T, K, H], w [T, K], shared_y or None) -> out [T, H] of out_dtype.
     A rank without tokens calls only `experts` (for the rows other ranks send it).
+    status() -> the first device-side error code (MOE_E*) the latest calls recorded, MOE_OK if
+    none, clearing them (synchronises); None when the steps record none.
     """
     route: Callable
     experts: Callable
     shared: Optional[Callable]
     combine: Callable
     out_dtype: torch.dtype = torch.float32
+    status: Optional[Callable] = None
 
 
 def placement_by_usage(order: torch.Tensor, n_ranks: int) -> tuple[torch.Tensor, torch.Tensor]:
@@ -179,11 +184,13 @@ def ep_cuda_compute(w_router: torch.Tensor, bias: torch.Tensor, cfg, routed, sha
     else:
         raise ValueError("routed experts: all E, or this rank's E / n_ranks")
 
+    last = {}  # each step's latest workspace: the kernels record device-side errors there
+
     def route(x):
         T = x.shape[0]
         idx = torch.empty(T, cfg.top_k, dtype=torch.int32, device=x.device)
         w = torch.empty(T, cfg.top_k, dtype=torch.float32, device=x.device)
-        ws = moe.workspace(moe.moe_route_workspace_bytes(T, cfg))
+        ws = last["route"] = moe.workspace(moe.moe_route_workspace_bytes(T, cfg))
         moe.moe_route(x, w_router, bias, cfg, idx, w, ws)
         return idx, w
 
@@ -197,14 +204,14 @@ def ep_cuda_compute(w_router: torch.Tensor, bias: torch.Tensor, cfg, routed, sha
         pair_slot = torch.empty(R, dtype=torch.int32, device=dev)
         moe.moe_union(local_idx.view(R, 1), per, n_unique, uniq, offsets, pair_tok, pair_slot)
         y = torch.empty(R, 1, local.hidden, dtype=torch.float32, device=dev)
-        ws = moe.workspace(moe.moe_expert_ffn_workspace_bytes(local, R, 1))
+        ws = last["experts"] = moe.workspace(moe.moe_expert_ffn_workspace_bytes(local, R, 1))
         moe.moe_expert_ffn_q(local, rows, 1, (n_unique, uniq, offsets, pair_tok, pair_slot), y, ws)
         return y.view(R, local.hidden)
 
     def shared_fn(x):
         T = x.shape[0]
         y = torch.empty(T, 1, shared.hidden, dtype=torch.float32, device=x.device)
-        ws = moe.workspace(moe.moe_expert_ffn_workspace_bytes(shared, T, 1))
+        ws = last["shared"] = moe.workspace(moe.moe_expert_ffn_workspace_bytes(shared, T, 1))
         moe.moe_expert_ffn_q(shared, x, 1, None, y, ws)
         return y.view(T, shared.hidden)
 
@@ -214,4 +221,8 @@ def ep_cuda_compute(w_router: torch.Tensor, bias: torch.Tensor, cfg, routed, sha
         moe.moe_combine(y_pairs, w, shared_y, out)
         return out
 
-    return EPCompute(route, experts, shared_fn if shared is not None else None, combine, out_dtype)
+    def status():
+        codes = [moe.moe_workspace_status(ws) for ws in last.values()]
+        return next((c for c in codes if c != moe.MOE_OK), moe.MOE_OK)
+
+    return EPCompute(route, experts, shared_fn if shared is not None else None, combine, out_dtype, status)

@@ -14,6 +14,7 @@ import torch.distributed as dist
 
 import synth
 from oracle import oracle as O
+from quantized_mixture_experts_sigmoid_b200 import moe
 from quantized_mixture_experts_sigmoid_b200.expert_parallel import ep_cuda_compute, ep_forward
 from synth.device import device_layer, to_dev_bf16
 from tests.helpers import layer_inputs, oracle_experts
@@ -49,7 +50,7 @@ def test_ep_one_rank_equals_oracle(name, one_rank_group):
     x, W, b = layer_inputs(sh)
     compute = ep_cuda_compute(dev["W"], dev["bias"], cfg, dev["routed"], dev["shared"], out_dtype=torch.float32)
     out = ep_forward(to_dev_bf16(x), sh.E, compute)
-    torch.cuda.synchronize()
+    assert compute.status() == moe.MOE_OK  # no device-side error recorded by the rank's steps
     routed = oracle_experts(sh, range(sh.E))
     shared = oracle_experts(sh, [0], shared=True)
     of, _, idx, _ = O.layer_forward(x, W, b, sh.n_group, sh.topk_group, sh.top_k, sh.rsf, routed, shared, top_p)
