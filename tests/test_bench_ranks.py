@@ -59,6 +59,15 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+    # the line carries the contract's keys, on the CUDA arm's metric and workload
+    for key in ("metric", "unit", "higher_is_better", "steps", "warmup", "ms_per_step", "config", "cpu_baseline", "e2e"):
+        assert key in rec, key
+    assert rec["unit"] == "tokens/s" and rec["higher_is_better"] is True and "workload" in rec["config"]
+    cb = rec["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == rec["value"]
+    e2e = rec["e2e"]
+    assert e2e["value"] == rec["value"] and e2e["unit"] == rec["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
 
 def test_layer_roofline_takes_the_slower_of_stream_and_contraction():
